@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Benchmark of the QK-Norm / FlashNorm hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch of synthetic input that is
+already resident in HBM:
+
+* QK-Norm workloads (default ``long_context``: 131072 tokens, q = k = 4096,
+  bf16, n_seg = 8): one ``qknorm_fused`` launch normalising every q row and k
+  row.  Metric: tokens/s; the roofline is HBM bandwidth.
+* ``flashnorm_proj`` (x[8192,4096] x W'[4096,12288], bf16): the 1/rms row
+  statistic plus the tcgen05 GEMM with the scaling epilogue.  Metric:
+  tokens/s; the roofline is the bf16 tensor-core peak.  The unfused
+  comparison (RMSNorm, then cuBLAS on the normalised x) is timed beside it.
+
+Multi-GPU (torchrun, one rank per GPU): tokens are independent, so every rank
+processes its own batch (weak scaling, no collective on the data path); the
+time is the max over ranks of the device-timed region and ``value`` counts the
+tokens of all ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
+bounded sample of the same workload per step), on rank 0 only.
+
+Rank 0 prints exactly one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+QK_DEFAULT = "long_context"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default depends on workload)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=QK_DEFAULT,
+                    choices=["tiny", "decode", "prefill_gqa", "long_context", "flashnorm_proj"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--strong", action="store_true",
+                    help="split one batch over the ranks (strong scaling) instead of one batch per rank")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline work budget")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def source_digest(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key: str, workload: str, src_paths):
+    """DRAM bytes per launch from a committed ncu capture, or None if absent or stale."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    e = t.get(kernel_key, {}).get(workload)
+    if not e or e.get("source_digest") != source_digest(src_paths):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.path = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.6)
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self, gpu_index=None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    rows.append({"ts": ts, "index": int(parts[1]), "sm": float(parts[2]), "max": float(parts[3]),
+                                 "power": float(parts[4]) if parts[4] not in ("[N/A]", "") else None,
+                                 "hw_slowdown": parts[6], "hw_thermal": parts[7], "sw_thermal": parts[8],
+                                 "sw_power_cap": parts[9]})
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        if gpu_index is not None:
+            sel = [r for r in rows if r["index"] == gpu_index] or rows
+        else:
+            sel = rows
+        # samples inside the timed window (1 s timestamp resolution)
+        win = [r for r in sel if self.t0 is not None and math.floor(self.t0) <= r["ts"] <= math.ceil(self.t1)]
+        if not win:
+            win = sel
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        for r in win:
+            for k in ("hw_slowdown", "hw_thermal", "sw_thermal", "sw_power_cap"):
+                if r[k].lower() == "active":
+                    reasons.add({"hw_thermal": "hw_thermal_slowdown", "sw_thermal": "sw_thermal_slowdown"}.get(k, k))
+        return {"sm_mhz": statistics.median(r["sm"] for r in win), "sm_max_mhz": max(r["max"] for r in win),
+                "reasons": sorted(reasons), "samples": len(win)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return rank, world, local, pg
+
+
+def max_over_ranks(value: float, pg):
+    from rmsnorm_qknorm_b200 import dist as qdist
+    return qdist.max_over_ranks(value, device="cuda") if pg is not None else value
+
+
+def barrier(pg):
+    import torch
+    torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+
+
+# -------------------------------------------------------------------- CPU baseline (oracle)
+
+
+def cpu_baseline_qknorm(inp_host, budget_s: float):
+    """fp64 oracle on a bounded sample of the workload's rows; returns a cpu_baseline dict."""
+    import oracle
+    q, k, wq, wk, eps = inp_host["q"], inp_host["k"], inp_host["wq"], inp_host["wk"], inp_host["eps"]
+    T = q.shape[0]
+    wq64, wk64 = oracle.as_f64(wq), oracle.as_f64(wk)
+    chunk = min(T, 1024)
+    done, elapsed, pos = 0, 0.0, 0
+    while elapsed < budget_s:
+        n = min(chunk, T - pos)
+        q64 = oracle.as_f64(q[pos:pos + n])
+        k64 = oracle.as_f64(k[pos:pos + n])
+        t0 = time.perf_counter()
+        oracle.rmsnorm(q64, wq64, eps)
+        oracle.rmsnorm(k64, wk64, eps)
+        elapsed += time.perf_counter() - t0
+        done += n
+        pos = (pos + n) % T
+        if elapsed < budget_s / 8:
+            chunk = min(T, chunk * 2)
+    return {"value": done / elapsed, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{done} token rows (q and k) cycling over the first {T} tokens of the workload, "
+                      f"fp64 C oracle, OpenMP over rows, {elapsed:.1f} s of CPU work"}
+
+
+def cpu_baseline_flashnorm(inp_host, budget_s: float):
+    import oracle
+    x, w, Wm, eps = inp_host["x"], inp_host["w"], inp_host["W"], inp_host["eps"]
+    M = x.shape[0]
+    w64, W64 = oracle.as_f64(w), oracle.as_f64(Wm)
+    done, elapsed, chunk, pos = 0, 0.0, 8, 0
+    while elapsed < budget_s:
+        n = min(chunk, M - pos)
+        x64 = oracle.as_f64(x[pos:pos + n])
+        t0 = time.perf_counter()
+        oracle.norm_then_project(x64, w64, W64, eps)
+        elapsed += time.perf_counter() - t0
+        done += n
+        pos = (pos + n) % M
+        if elapsed < budget_s / 8:
+            chunk = min(M, chunk * 2)
+    return {"value": done / elapsed, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{done} rows of x (cycling over {M} rows) through RMSNorm then the "
+                      f"[4096 x 12288] projection, fp64 C oracle, {elapsed:.1f} s of CPU work"}
+
+
+# ------------------------------------------------------------------------ reference arm
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from rmsnorm_qknorm_b200 import workloads as W
+    steps = args.steps if args.steps is not None else 5
+    if args.workload == "flashnorm_proj":
+        wl = W.FLASHNORM_WORKLOAD
+        inp = W.make_flashnorm_inputs(seed=0, M=64)
+        fn = lambda: cpu_baseline_flashnorm(inp, 4.0)  # noqa: E731
+        metric = "FlashNorm norm-then-project tokens/s (fp64 CPU oracle)"
+        cfg = {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N}
+    else:
+        wl = W.QKNORM_WORKLOADS[args.workload]
+        inp = W.make_qknorm_inputs(wl, seed=0, tokens=min(wl.tokens, 8192))
+        fn = lambda: cpu_baseline_qknorm(inp, 4.0)  # noqa: E731
+        metric = "QK-Norm tokens/s (fp64 CPU oracle)"
+        cfg = {"workload": wl.name, "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk, "n_seg": wl.n_seg}
+    for _ in range(args.warmup):
+        fn()
+    vals = [fn() for _ in range(steps)]
+    value = statistics.median(v["value"] for v in vals)
+    last = vals[-1]
+    print(json.dumps({
+        "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- our arm
+
+
+def time_launches(fn, steps, stream):
+    """Runs fn() `steps` times; returns (total ms, per-launch ms list) from CUDA events on `stream`."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        fn(i)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    t_end.synchronize()
+    return t_start.elapsed_time(t_end), [a.elapsed_time(b) for a, b in ev]
+
+
+def run_qknorm(args, rank, world, local, pg):
+    import torch
+    import rmsnorm_qknorm_b200 as qk
+    from rmsnorm_qknorm_b200 import workloads as W
+    qk.load_library()
+    from rmsnorm_qknorm_b200 import dist as qdist
+    wl = W.QKNORM_WORKLOADS[args.workload]
+    steps = args.steps if args.steps is not None else (2000 if wl.tokens >= 100000 else 5000)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    if args.strong:
+        r0, r1 = qdist.shard_rows(wl.tokens, rank, world)
+        my_tokens, global_tokens = r1 - r0, wl.tokens
+    else:
+        my_tokens, global_tokens = wl.tokens, world * wl.tokens
+    per_set = wl.algorithmic_bytes(my_tokens)
+    nsets = 1 if per_set > 2 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_set))
+    sets = []
+    for s in range(nsets):
+        inp = W.make_qknorm_inputs(wl, seed=qdist.rank_seed(s, rank), device=dev, tokens=my_tokens)
+        inp["q_out"] = torch.empty_like(inp["q"])
+        inp["k_out"] = torch.empty_like(inp["k"])
+        sets.append(inp)
+
+    def step(i):
+        s = sets[i % nsets]
+        qk.qknorm_fused(s["q"], s["k"], s["wq"], s["wk"], wl.eps, wl.n_seg, q_out=s["q_out"], k_out=s["k_out"])
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    barrier(pg)
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+        clocks.mark(True)
+    total_ms, launch_ms = time_launches(step, steps, stream)
+    if clocks:
+        clocks.mark(False)
+    barrier(pg)
+    total_ms = max_over_ranks(total_ms, pg)
+    avg_launch_ms = max_over_ranks(statistics.mean(launch_ms), pg)
+    clk = clocks.stop(gpu_index=local) if clocks else None
+
+    ms_per_step = total_ms / steps
+    value = global_tokens / (ms_per_step * 1e-3)
+    pk, pk_kind = peaks()
+    achieved = per_set / (avg_launch_ms * 1e-3) / 1e9
+    src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh"]
+    traffic = traffic_for("rownorm_vec_kernel", wl.name, src)
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        s = sets[0]
+        hq = s["q"].cpu().pin_memory()
+        hk = s["k"].cpu().pin_memory()
+        oq = torch.empty_like(hq).pin_memory()
+        ok = torch.empty_like(hk).pin_memory()
+        dq, dk = torch.empty_like(s["q"]), torch.empty_like(s["k"])
+
+        def e2e_step(_i):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            qo, ko = qk.qknorm_fused(dq, dk, s["wq"], s["wk"], wl.eps, wl.n_seg, q_out=s["q_out"], k_out=s["k_out"])
+            oq.copy_(qo, non_blocking=True)
+            ok.copy_(ko, non_blocking=True)
+
+        e2e_step(0)
+        barrier(pg)
+        e_ms, _ = time_launches(e2e_step, args.e2e_steps, stream)
+        barrier(pg)
+        e_ms = max_over_ranks(e_ms, pg)
+        h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size()
+        e2e = {"value": global_tokens / (e_ms / args.e2e_steps * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
+               "note": "pinned host q,k -> device, qknorm_fused, device -> pinned host outputs, per step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = W.make_qknorm_inputs(wl, seed=0, device="cpu", tokens=min(wl.tokens, 65536))
+        cpu = cpu_baseline_qknorm(host, args.cpu_seconds)
+
+    if rank == 0:
+        out = {
+            "metric": "QK-Norm tokens/s and achieved HBM GB/s (% of B200 roofline) on 1 GPU",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if args.strong else "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "tokens_per_gpu": my_tokens, "global_tokens": global_tokens,
+                       "dq": wl.dq, "dk": wl.dk, "n_seg": wl.n_seg, "eps": wl.eps,
+                       "parallelism": f"dp{world} (token batches, no collective)",
+                       "l2": ("inputs larger than L2" if nsets == 1 else
+                              f"{nsets} rotating input sets totalling {nsets * per_set / 1e6:.0f} MB > L2")},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                         "kernel": "rownorm_vec_kernel",
+                         "algorithmic_bytes_per_launch": per_set,
+                         "avg_launch_us": avg_launch_ms * 1e3,
+                         "peak_source": f"{pk_kind} HBM copy bandwidth",
+                         "frac_of_8TBs": achieved / 8000.0},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": steps,
+            "clocks": clk,
+        }
+        print(json.dumps(out), flush=True)
+
+
+def run_flashnorm(args, rank, world, local, pg):
+    import torch
+    import rmsnorm_qknorm_b200 as qk
+    from rmsnorm_qknorm_b200 import workloads as W
+    qk.load_library()
+    wl = W.FLASHNORM_WORKLOAD
+    steps = args.steps if args.steps is not None else 200
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    from rmsnorm_qknorm_b200 import dist as qdist
+    inp = W.make_flashnorm_inputs(seed=qdist.rank_seed(0, rank), device=dev)
+    x, w, Wm = inp["x"], inp["w"], inp["W"]
+    Wf = qk.flashnorm_fold_weights(w, Wm)
+    y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
+    inv = torch.empty(wl.M, dtype=torch.float32, device=dev)
+
+    def step(_i):
+        qk.flashnorm_proj(x, Wf, wl.eps, inv_rms_out=inv, out=y)
+
+    def gemm_only(_i):
+        qk.flashnorm_proj(x, Wf, wl.eps, inv_rms=inv, out=y)
+
+    # unfused comparison: RMSNorm kernel writing normalised x, then cuBLAS with the original W
+    xn = torch.empty_like(x)
+
+    def unfused(_i):
+        qk.qknorm_fused(x, None, w, None, wl.eps, 1, q_out=xn)
+        torch.matmul(xn, Wm, out=y)
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+        gemm_only(i)
+        unfused(i)
+    barrier(pg)
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+        clocks.mark(True)
+    total_ms, _ = time_launches(step, steps, stream)
+    gemm_total, gemm_ms = time_launches(gemm_only, steps, stream)
+    if clocks:
+        clocks.mark(False)
+    unf_ms, _ = time_launches(unfused, steps, stream)
+    barrier(pg)
+    total_ms = max_over_ranks(total_ms, pg)
+    avg_gemm = max_over_ranks(statistics.mean(gemm_ms), pg)
+    unf_ms = max_over_ranks(unf_ms, pg)
+    clk = clocks.stop(gpu_index=local) if clocks else None
+    ms_per_step = total_ms / steps
+    value = world * wl.M / (ms_per_step * 1e-3)
+    pk, pk_kind = peaks()
+    tflops = wl.flops() / (avg_gemm * 1e-3) / 1e12
+    src = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh"]
+
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = x.cpu().pin_memory()
+        hy = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
+        dx = torch.empty_like(x)
+
+        def e2e_step(_i):
+            dx.copy_(hx, non_blocking=True)
+            qk.flashnorm_proj(dx, Wf, wl.eps, inv_rms_out=inv, out=y)
+            hy.copy_(y, non_blocking=True)
+
+        e2e_step(0)
+        barrier(pg)
+        e_ms, _ = time_launches(e2e_step, args.e2e_steps, stream)
+        barrier(pg)
+        e_ms = max_over_ranks(e_ms, pg)
+        e2e = {"value": world * wl.M / (e_ms / args.e2e_steps * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2,
+               "note": "pinned host x -> device, flashnorm_proj, device -> pinned host y, per step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = W.make_flashnorm_inputs(seed=0, device="cpu", M=256)
+        cpu = cpu_baseline_flashnorm(host, args.cpu_seconds)
+
+    if rank == 0:
+        print(json.dumps({
+            "metric": "FlashNorm norm-then-project tokens/s and tensor-core TFLOP/s (% of bf16 peak) on 1 GPU",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "eps": wl.eps,
+                       "parallelism": f"dp{world} (token batches, no collective)",
+                       "l2": "inputs larger than L2 (x 67 MB + W' 101 MB)"},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / pk["bf16_tflops"], "kernel": "flashnorm_gemm_kernel",
+                         "traffic": traffic_for("flashnorm_gemm_kernel", wl.name, src),
+                         "avg_launch_us": avg_gemm * 1e3, "flops_per_launch": wl.flops(),
+                         "peak_source": f"{pk_kind} cuBLAS bf16 burst"},
+            "comparison": {"unfused_ms_per_step": unf_ms / steps, "fused_ms_per_step": ms_per_step,
+                           "speedup_vs_unfused": (unf_ms / steps) / ms_per_step,
+                           "unfused": "qknorm_fused RMSNorm writing x_hat, then torch.matmul (cuBLAS) with W"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * steps, "clocks": clk,
+        }), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    rank, world, local, pg = dist_setup(args)
+    try:
+        if args.workload == "flashnorm_proj":
+            run_flashnorm(args, rank, world, local, pg)
+        else:
+            run_qknorm(args, rank, world, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * qknorm.h -- C ABI of libqknorm.so: layerwise QK-Norm with segment-wise
+ * scalar statistics, and the FlashNorm fold + deferred-normalisation
+ * projection, as hand-written CUDA kernels for B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *   keeps no pointer after the call returns.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *   stream).  Work is enqueued asynchronously on it; nothing synchronises.
+ * - Arguments are validated on the host before anything is launched.  A
+ *   failed validation returns a nonzero qkn_status, launches nothing, and
+ *   leaves a message in qkn_last_error() (thread-local).
+ * - QKN_ERR_CUDA reports an error returned by the CUDA runtime for this
+ *   call's launches (cudaGetLastError right after them); errors raised later
+ *   by the device surface at the caller's next synchronisation, as usual.
+ * - Rows are independent; an empty problem (zero rows) is valid, launches
+ *   nothing and accepts NULL data pointers (an empty tensor may have no
+ *   storage).  NaN / Inf inputs propagate to the rows that contain them.
+ * - Results are deterministic: the same inputs give bitwise-equal outputs on
+ *   every call (fixed reduction orders, no atomics).
+ */
+#ifndef QKNORM_H
+#define QKNORM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QKN_API __attribute__((visibility("default")))
+#else
+#define QKN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QKN_OK = 0,
+    QKN_ERR_NULL = 1,        /* a required pointer is NULL */
+    QKN_ERR_SHAPE = 2,       /* negative size, zero width, leading dimension < width,
+                                width not a multiple of n_seg, n_seg out of range,
+                                or a size rule of the entry point not met */
+    QKN_ERR_DTYPE = 3,       /* unknown qkn_dtype or a combination not offered */
+    QKN_ERR_EPS = 4,         /* eps negative, NaN or infinite */
+    QKN_ERR_ALIGN = 5,       /* an alignment the entry point requires is not met */
+    QKN_ERR_CUDA = 6,        /* the CUDA runtime reported an error for this call */
+    QKN_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up */
+    QKN_ERR_UNSUPPORTED = 8  /* well-formed request outside what this build implements */
+} qkn_status;
+
+typedef enum {
+    QKN_F32 = 0,   /* IEEE binary32 */
+    QKN_BF16 = 1   /* bfloat16 (1 sign, 8 exponent, 7 fraction bits) */
+} qkn_dtype;
+
+/* Largest number of segments (emulated tensor-parallel shards) per row. */
+#define QKN_MAX_SEG 64
+
+/*
+ * qknorm_fused -- layerwise QK-Norm of the query and key rows in ONE launch.
+ *
+ * Defined by: SwiftQK (montaan.com 2608.09160), abstract -- QK-Norm is an
+ * RMSNorm whose factor depends on each token's full q (resp. k) vector; under
+ * tensor parallelism every shard contributes a scalar partial sum of squares
+ * and only these scalars are combined.  Here the n_seg shards are emulated on
+ * one GPU as n_seg contiguous equal segments of each row:
+ *   S_j  = sum over segment j of x_i^2                       (fp32)
+ *   S    = ((S_0 + S_1) + S_2) + ... + S_{n_seg-1}            (fixed order)
+ *   inv  = 1 / sqrt(S / d + eps)
+ *   y_i  = (x_i * inv) * w_i, rounded once to the activation dtype.
+ *
+ * q      [T][dq] activations, row pitch ldq elements (ldq >= dq)
+ * k      [T][dk] activations, row pitch ldk; dk == 0 normalises q only (k, wk
+ *        and k_out are then ignored)
+ * wq, wk [dq], [dk] weights, dtype `wdt` (may differ from `act`)
+ * q_out, k_out  outputs [T][d] with pitches ldq_out, ldk_out; pass q_out ==
+ *        NULL (resp. k_out == NULL) to normalise in place, in which case the
+ *        input pitch is used and the ld*_out argument is ignored
+ * act    QKN_F32 or QKN_BF16 (inputs and outputs); statistics are always fp32
+ * eps    >= 0 and finite; a zero row with eps == 0 gives NaN (0/0), not an error
+ * n_seg  1 .. QKN_MAX_SEG; dq and dk must both be multiples of n_seg
+ *
+ * Alignment: any element-aligned pointers and pitches are accepted.  When
+ * every row start is 16-byte aligned and each segment is a whole number of
+ * 16-byte chunks, the vectorised kernel runs; otherwise a slower element-wise
+ * kernel computes the same result.
+ */
+QKN_API qkn_status qknorm_fused(const void *q, const void *k,
+                                const void *wq, const void *wk,
+                                void *q_out, void *k_out,
+                                int64_t T, int64_t dq, int64_t dk,
+                                int64_t ldq, int64_t ldk,
+                                int64_t ldq_out, int64_t ldk_out,
+                                qkn_dtype act, qkn_dtype wdt,
+                                float eps, int n_seg, void *stream);
+
+/*
+ * rmsnorm_partial_stats -- the per-shard scalar statistics on their own.
+ *
+ * Defined by: SwiftQK, abstract -- the scalar partial sums of squares that
+ * the shards exchange instead of the full activation vectors.
+ *   partial[r][j] = sum_{i in [j*d/n_seg, (j+1)*d/n_seg)} x[r][i]^2  (fp32)
+ *
+ * x        [rows][d], pitch ld >= d, dtype `act` (QKN_F32 or QKN_BF16)
+ * partial  [rows][n_seg] fp32, contiguous, written completely
+ * n_seg    1 .. QKN_MAX_SEG, d % n_seg == 0
+ * The summation order inside a segment is fixed for a given row width and
+ * n_seg, so repeated calls give bitwise-equal partials.
+ */
+QKN_API qkn_status rmsnorm_partial_stats(const void *x, int64_t rows, int64_t d,
+                                         int64_t ld, qkn_dtype act, int n_seg,
+                                         float *partial, void *stream);
+
+/*
+ * flashnorm_fold_weights -- fold the RMSNorm weights into the next linear
+ * layer (offline).
+ *
+ * Defined by: FlashNorm (Graef, arXiv 2024), abstract, item (i): the
+ * normalisation weights disappear into the following weight matrix,
+ *   W'[k][n] = w[k] * W[k][n]   computed in fp32, rounded once to bf16.
+ *
+ * w         [K], dtype `wdt` (QKN_F32 or QKN_BF16)
+ * W         [K][N] bf16, row-major (N contiguous)
+ * W_folded  bf16 output, [K][N] row-major when out_k_major == 0, or the
+ *           transposed [N][K] (K contiguous) when out_k_major == 1 -- the
+ *           layout flashnorm_proj reads
+ * W_folded must not overlap W.
+ */
+QKN_API qkn_status flashnorm_fold_weights(const void *w, const void *W, void *W_folded,
+                                          int64_t K, int64_t N, qkn_dtype wdt,
+                                          int out_k_major, void *stream);
+
+/*
+ * flashnorm_proj -- RMSNorm followed by a linear layer, computed as
+ * FlashNorm's deferred normalisation: a bf16 tensor-core GEMM on the raw x
+ * with the folded weights, the scalar 1/rms(x) applied in the epilogue.
+ *
+ * Defined by: FlashNorm, abstract, item (ii): the scalar RMS normalisation is
+ * moved to the matmul output, so RMS and matmul can run in parallel.
+ *   inv[m]  = 1 / sqrt(sum_k x[m][k]^2 / K + eps)               (fp32)
+ *   y[m][n] = inv[m] * sum_k x[m][k] * W'[n][k]   fp32 accumulate, bf16 out
+ *
+ * x          [M][K] bf16, row-major (K contiguous)
+ * W_folded   [N][K] bf16 (K contiguous, out_k_major == 1 of the fold);
+ *            w_k_major must be 1 (0 returns QKN_ERR_UNSUPPORTED)
+ * y          [M][N] bf16, row-major
+ * inv_rms    optional [M] fp32 precomputed 1/rms; NULL = compute from x and eps
+ * inv_rms_out optional [M] fp32 that receives the 1/rms used (when inv_rms is
+ *            NULL); when both are NULL the library takes stream-ordered
+ *            scratch of M floats from the CUDA memory pool for the call
+ * Sizes: M, N, K >= 1; K and N multiples of 8.  Pointers 16-byte aligned.
+ * y must not overlap x or W_folded.
+ */
+QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y,
+                                  int64_t M, int64_t N, int64_t K, int w_k_major,
+                                  float eps, const float *inv_rms, float *inv_rms_out,
+                                  void *stream);
+
+/*
+ * qkn_check_device -- synchronises `stream`, then reads and clears the
+ * current device's error word.  Returns QKN_ERR_TIMEOUT when a bounded
+ * device-side wait of an earlier launch (the projection kernel's mbarrier
+ * waits give up after 2 s) recorded a failure, QKN_ERR_CUDA when the
+ * synchronisation itself failed, QKN_OK otherwise.  Not part of the page's
+ * method: it is the host-visible end of the kernels' bounded waits.
+ */
+QKN_API qkn_status qkn_check_device(void *stream);
+
+/* Message describing the last nonzero status returned on this host thread. */
+QKN_API const char *qkn_last_error(void);
+
+/* Library version string, e.g. "qknorm 0.1.0 sm_100a". */
+QKN_API const char *qkn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNORM_H */

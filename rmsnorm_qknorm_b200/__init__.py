@@ -1,1 +1,248 @@
-"""B200-native QK-Norm and FlashNorm (placeholder; the binding lands with the C ABI)."""
+"""B200-native layerwise QK-Norm and FlashNorm: Python binding of libqknorm.so.
+
+This module only marshals arguments: it checks tensor placement, reads
+pointers, pitches and the current CUDA stream from torch, and calls the C ABI
+declared in ``include/qknorm.h``.  Every step of the computation runs in the
+library's sm_100a kernels; there is no CPU or PyTorch fallback, and a missing
+library raises instead of degrading.
+
+Entry points (same names as the C ABI):
+
+* :func:`qknorm_fused` -- RMSNorm of every query row and key row in one launch,
+  statistics built from ``n_seg`` per-segment scalar partial sums combined in a
+  fixed order (SwiftQK's tensor-parallel statistic, emulated on one GPU).
+* :func:`rmsnorm_partial_stats` -- those per-segment partial sums on their own.
+* :func:`flashnorm_fold_weights` -- FlashNorm's W' = diag(w) W.
+* :func:`flashnorm_proj` -- y = (x W') * 1/rms(x), the deferred-normalisation
+  GEMM with the scaling in the epilogue.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "QKNormError",
+    "load_library",
+    "library_path",
+    "qknorm_fused",
+    "rmsnorm_partial_stats",
+    "flashnorm_fold_weights",
+    "flashnorm_proj",
+    "STATUS_NAMES",
+    "QKN_MAX_SEG",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libqknorm.so")
+_lock = threading.Lock()
+_lib = None
+
+QKN_MAX_SEG = 64
+QKN_F32, QKN_BF16 = 0, 1
+STATUS_NAMES = {
+    0: "QKN_OK", 1: "QKN_ERR_NULL", 2: "QKN_ERR_SHAPE", 3: "QKN_ERR_DTYPE", 4: "QKN_ERR_EPS",
+    5: "QKN_ERR_ALIGN", 6: "QKN_ERR_CUDA", 7: "QKN_ERR_TIMEOUT", 8: "QKN_ERR_UNSUPPORTED",
+}
+
+
+class QKNormError(RuntimeError):
+    """A nonzero qkn_status from the library, with its message."""
+
+    def __init__(self, fn: str, status: int, message: str):
+        self.status = status
+        self.status_name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{fn}: {self.status_name}: {message}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libqknorm.so (built by ``python -m rmsnorm_qknorm_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(
+                f"{_LIB_PATH} is missing: build it with `python -m rmsnorm_qknorm_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        p, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        lib.qknorm_fused.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, i64, i64, i64,
+                                     i32, i32, f32, i32, p]
+        lib.rmsnorm_partial_stats.argtypes = [p, i64, i64, i64, i32, i32, p, p]
+        lib.flashnorm_fold_weights.argtypes = [p, p, p, i64, i64, i32, i32, p]
+        lib.flashnorm_proj.argtypes = [p, p, p, i64, i64, i64, i32, f32, p, p, p]
+        for f in ("qknorm_fused", "rmsnorm_partial_stats", "flashnorm_fold_weights",
+                  "flashnorm_proj"):
+            getattr(lib, f).restype = ctypes.c_int
+        lib.qkn_last_error.restype = ctypes.c_char_p
+        lib.qkn_last_error.argtypes = []
+        lib.qkn_version.restype = ctypes.c_char_p
+        lib.qkn_version.argtypes = []
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        msg = load_library().qkn_last_error().decode(errors="replace")
+        raise QKNormError(fn, status, msg)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return QKN_F32
+    if t == torch.bfloat16:
+        return QKN_BF16
+    raise TypeError(f"unsupported dtype {t}; expected torch.float32 or torch.bfloat16")
+
+
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    return t
+
+
+def _rows(t: torch.Tensor, name: str):
+    _cuda(t, name)
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be 2-D with unit stride along the row")
+    return t.shape[0], t.shape[1], max(t.stride(0), t.shape[1])
+
+
+def _vec(t: torch.Tensor, name: str, n: int):
+    _cuda(t, name)
+    if t.dim() != 1 or t.shape[0] != n or (n > 1 and t.stride(0) != 1):
+        raise ValueError(f"{name} must be a contiguous 1-D tensor of length {n}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def qknorm_fused(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
+                 wk: torch.Tensor | None, eps: float = 1e-6, n_seg: int = 1, *,
+                 q_out: torch.Tensor | None = None, k_out: torch.Tensor | None = None,
+                 inplace: bool = False, stream=None):
+    """QK-Norm of q [T, dq] and k [T, dk] (k may be None) in one launch.
+
+    Returns ``(q_out, k_out)``.  With ``inplace=True`` the inputs are
+    overwritten and returned; otherwise outputs are allocated unless given.
+    Row pitches are taken from the tensors' strides (views of a fused QKV
+    buffer work without copies).
+    """
+    T, dq, ldq = _rows(q, "q")
+    act = _dtype_code(q.dtype)
+    _vec(wq, "wq", dq)
+    wdt = _dtype_code(wq.dtype)
+    if k is not None:
+        Tk, dk, ldk = _rows(k, "k")
+        if Tk != T or k.dtype != q.dtype:
+            raise ValueError("k must have q's row count and dtype")
+        if wk is None:
+            raise ValueError("wk is required with k")
+        _vec(wk, "wk", dk)
+        if wk.dtype != wq.dtype:
+            raise ValueError("wk must have wq's dtype")
+    else:
+        dk, ldk = 0, 0
+    if inplace:
+        q_out_t, k_out_t = q, k
+        q_ptr_out = k_ptr_out = None
+        ldq_o, ldk_o = ldq, ldk
+    else:
+        q_out_t = q_out if q_out is not None else torch.empty((T, dq), dtype=q.dtype, device=q.device)
+        _, _, ldq_o = _rows(q_out_t, "q_out")
+        q_ptr_out = q_out_t.data_ptr()
+        if k is not None:
+            k_out_t = k_out if k_out is not None else torch.empty((T, dk), dtype=k.dtype, device=k.device)
+            _, _, ldk_o = _rows(k_out_t, "k_out")
+            k_ptr_out = k_out_t.data_ptr()
+        else:
+            k_out_t, k_ptr_out, ldk_o = None, None, 0
+    lib = load_library()
+    st = lib.qknorm_fused(q.data_ptr(), k.data_ptr() if k is not None else None,
+                          wq.data_ptr(), wk.data_ptr() if k is not None else None,
+                          q_ptr_out, k_ptr_out, T, dq, dk, ldq, ldk, ldq_o, ldk_o,
+                          act, wdt, float(eps), int(n_seg), _stream(stream))
+    _check("qknorm_fused", st)
+    return q_out_t, k_out_t
+
+
+def rmsnorm_partial_stats(x: torch.Tensor, n_seg: int, *, out: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    """Per-row sums of squares of n_seg contiguous segments: fp32 [rows, n_seg]."""
+    rows, d, ld = _rows(x, "x")
+    act = _dtype_code(x.dtype)
+    if out is None:
+        out = torch.empty((rows, n_seg), dtype=torch.float32, device=x.device)
+    elif out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != (rows, n_seg):
+        raise ValueError("out must be a contiguous fp32 tensor of shape [rows, n_seg]")
+    st = load_library().rmsnorm_partial_stats(x.data_ptr(), rows, d, ld, act, int(n_seg),
+                                              _cuda(out, "out").data_ptr(), _stream(stream))
+    _check("rmsnorm_partial_stats", st)
+    return out
+
+
+def flashnorm_fold_weights(w: torch.Tensor, W: torch.Tensor, *, k_major: bool = True,
+                           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """FlashNorm fold W' = diag(w) W of W [K, N] (bf16); [N, K] when k_major else [K, N]."""
+    _cuda(W, "W")
+    if W.dim() != 2 or not W.is_contiguous() or W.dtype != torch.bfloat16:
+        raise ValueError("W must be a contiguous bf16 [K, N] tensor")
+    K, N = W.shape
+    _vec(w, "w", K)
+    shape = (N, K) if k_major else (K, N)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=W.device)
+    elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != torch.bfloat16:
+        raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
+    st = load_library().flashnorm_fold_weights(w.data_ptr(), W.data_ptr(), _cuda(out, "out").data_ptr(),
+                                               K, N, _dtype_code(w.dtype), int(bool(k_major)),
+                                               _stream(stream))
+    _check("flashnorm_fold_weights", st)
+    return out
+
+
+def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *,
+                   inv_rms: torch.Tensor | None = None, inv_rms_out: torch.Tensor | None = None,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [M, N] = (x [M, K] @ W_folded[N, K]^T) * 1/rms(x), bf16 in/out, fp32 accumulate."""
+    _cuda(x, "x")
+    _cuda(W_folded, "W_folded")
+    if x.dim() != 2 or not x.is_contiguous() or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a contiguous bf16 [M, K] tensor")
+    if W_folded.dim() != 2 or not W_folded.is_contiguous() or W_folded.dtype != torch.bfloat16:
+        raise ValueError("W_folded must be a contiguous bf16 [N, K] tensor")
+    M, K = x.shape
+    N, K2 = W_folded.shape
+    if K2 != K:
+        raise ValueError(f"W_folded is [{N}, {K2}] but x has K={K}")
+    for name, t in (("inv_rms", inv_rms), ("inv_rms_out", inv_rms_out)):
+        if t is not None:
+            _vec(t, name, M)
+            if t.dtype != torch.float32:
+                raise ValueError(f"{name} must be fp32")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif tuple(out.shape) != (M, N) or not out.is_contiguous() or out.dtype != torch.bfloat16:
+        raise ValueError("out must be a contiguous bf16 [M, N] tensor")
+    st = load_library().flashnorm_proj(
+        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, N, K, 1, float(eps),
+        inv_rms.data_ptr() if inv_rms is not None else None,
+        inv_rms_out.data_ptr() if inv_rms_out is not None else None, _stream(stream))
+    _check("flashnorm_proj", st)
+    return out

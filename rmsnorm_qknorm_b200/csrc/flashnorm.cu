@@ -1,0 +1,515 @@
+// FlashNorm (Graef, arXiv 2024), abstract: RMSNorm followed by a linear layer,
+// reformulated exactly as
+//   (i)  W' = diag(w) W                       -- flashnorm_fold_weights (offline)
+//   (ii) y  = (x W') * 1/rms(x)               -- flashnorm_proj
+// The projection is a dense contraction, so it runs on the 5th-generation
+// tensor cores: a persistent, warp-specialised kernel in which one warp moves
+// 128x64 / 256x64 bf16 tiles with TMA into a ring of shared-memory stages, one
+// thread issues tcgen05.mma into a double-buffered fp32 accumulator in tensor
+// memory, and four epilogue warps read the accumulator back (tcgen05.ld),
+// multiply each row by its 1/rms and store bf16.  The 1/rms vector comes from
+// a small row-statistics kernel (or from the caller).
+#include <cuda.h>
+#include <math.h>
+
+#include "qkn_common.cuh"
+
+namespace qkn {
+
+// Set by any bounded device-side wait that gave up; read by qkn_check_device.
+__device__ int g_device_error = 0;
+
+// ============================================================== fold (i)
+
+// Row-major output: W'[k][n] = w[k] * W[k][n], 8 bf16 per thread.
+template <typename TW>
+__global__ void __launch_bounds__(256) fold_rowmajor_kernel(const TW *__restrict__ w,
+                                                            const __nv_bfloat16 *__restrict__ W,
+                                                            __nv_bfloat16 *__restrict__ Wf,
+                                                            int64_t K, int64_t N) {
+    const int64_t total = K * N;
+    for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x);
+         i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t k = i / N;
+        Wf[i] = __float2bfloat16_rn(to_f32<TW>(w[k]) * __bfloat162float(W[i]));
+    }
+}
+
+// Transposed output: W'[n][k] = w[k] * W[k][n] through a 64x64 shared tile.
+constexpr int kFoldTile = 64;
+
+template <typename TW>
+__global__ void __launch_bounds__(256) fold_transpose_kernel(const TW *__restrict__ w,
+                                                             const __nv_bfloat16 *__restrict__ W,
+                                                             __nv_bfloat16 *__restrict__ Wf,
+                                                             int64_t K, int64_t N) {
+    __shared__ __nv_bfloat16 tile[kFoldTile][kFoldTile + 2];
+    const int64_t k0 = (int64_t)blockIdx.y * kFoldTile, n0 = (int64_t)blockIdx.x * kFoldTile;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
+    for (int r = ty; r < kFoldTile; r += 4) {
+        const int64_t k = k0 + r, n = n0 + tx;
+        if (k < K && n < N)
+            tile[r][tx] = __float2bfloat16_rn(to_f32<TW>(w[k]) * __bfloat162float(W[k * N + n]));
+    }
+    __syncthreads();
+    for (int r = ty; r < kFoldTile; r += 4) {
+        const int64_t n = n0 + r, k = k0 + tx;
+        if (n < N && k < K) Wf[n * K + k] = tile[tx][r];
+    }
+}
+
+// ======================================================= row statistics
+
+// inv[m] = 1/sqrt(sum_k x[m][k]^2 / K + eps), one warp per row, 16-byte loads.
+// K is a multiple of 8 and rows are 16-byte aligned (checked by the caller).
+__global__ void __launch_bounds__(256) inv_rms_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                      float *__restrict__ inv, int64_t M, int64_t K,
+                                                      float eps) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= M) return;  // whole warp leaves together
+    const uint8_t *xr = reinterpret_cast<const uint8_t *>(x + row * K);
+    const int64_t nchunks = K / 8;
+    float s = 0.f;
+    for (int64_t c = lane; c < nchunks; c += 32) {
+        float f[8];
+        Chunk<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4 *>(xr + c * 16)), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s = fmaf(f[e], f[e], s);
+    }
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) inv[row] = rsqrtf(s / (float)K + eps);
+}
+
+// ===================================================== tcgen05 GEMM (ii)
+
+namespace gemm {
+
+constexpr int BM = 128, BN = 256, BK = 64;             // bf16: BK * 2 B = one 128-byte swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                    // 16 KiB
+constexpr int B_BYTES = BN * BK * 2;                    // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int UMMA_K = 16;                              // K of one kind::f16 MMA
+constexpr int ACC_COLS = BN;                            // fp32 accumulator: one column per n
+constexpr int TMEM_COLS = 2 * ACC_COLS;                 // double-buffered accumulator
+constexpr int THREADS = 192;                            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;      // 2 s: far above any tile's latency
+
+static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B (both
+// K-major), fp32 accumulator, M = 128, N = 256.
+constexpr uint32_t kInstrDesc = (1u << 4)                 // D format: f32
+                              | (1u << 7)                 // A format: bf16
+                              | (1u << 10)                // B format: bf16
+                              | (0u << 15) | (0u << 16)   // A, B K-major
+                              | ((uint32_t)(BN >> 3) << 17)
+                              | ((uint32_t)(BM >> 4) << 24);
+
+struct Args {
+    const float *inv_rms;   // [M]
+    __nv_bfloat16 *y;       // [M][N]
+    int M, N, K;
+    int m_blocks, n_blocks, k_blocks, num_tiles;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+                 ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up after
+// kWaitTimeoutNs, records the failure in g_device_error and returns false.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer() - t0 > kWaitTimeoutNs) {
+            atomicExch(&g_device_error, 1);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand stored as rows of 64
+// bf16 (128 bytes) with the 128-byte swizzle: groups of 8 rows are 1024 bytes
+// apart (stride byte offset); the leading byte offset is unused for this
+// layout and set to 1.  Stage buffers are 1024-byte aligned, so the base
+// offset field is 0.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;     // descriptor version for tcgen05
+    d |= (uint64_t)2u << 61;     // swizzle mode: 128 bytes
+    return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kInstrDesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns: thread i gets row (lane base + i).
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                      const Args g) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + STAGES;
+    uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);    // producer's arrive + TMA bytes
+            mbar_init(smem_u32(&empty[s]), 1);   // one tcgen05.commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&acc_full[a]), 1);   // one tcgen05.commit
+            mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrive per epilogue warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {  // whole warp: allocate the two accumulators in tensor memory
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
+            const int m_blk = tile % g.m_blocks, n_blk = tile / g.m_blocks;
+            for (int kb = 0; kb < g.k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u)) { ok = false; break; }
+                if (lane == 0) {
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    uint8_t *sa = smem + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(smem_u32(sa), &tmap_x, kb * BK, m_blk * BM, fb);
+                    tma_load_2d(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, n_blk * BN, fb);
+                }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+            for (int kb = 0; kb < g.k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase)) { ok = false; break; }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        // advancing K by 16 bf16 = 32 bytes inside the swizzle row
+                        umma_bf16(d_tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32),
+                                  (kb | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&empty[stage]));  // frees the stage once these MMAs read it
+                }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(smem_u32(&acc_full[acc]));  // accumulator ready
+            __syncwarp();
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2..5)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access: 32 * quarter ...
+        int it = 0;
+        for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++it) {
+            const int m_blk = tile % g.m_blocks, n_blk = tile / g.m_blocks;
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase)) break;
+            tc_fence_after();
+            const int row = m_blk * BM + quarter * 32 + lane;
+            const bool row_ok = row < g.M;
+            const float r = row_ok ? __ldg(g.inv_rms + row) : 0.f;
+            __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32cols(tbase + c * 32, v);
+                const int col0 = n_blk * BN + c * 32;
+                if (row_ok) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int col = col0 + j * 8;
+                        if (col < g.N) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * r, __uint_as_float(v[8 * j + 1]) * r);
+                            o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * r, __uint_as_float(v[8 * j + 3]) * r);
+                            o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * r, __uint_as_float(v[8 * j + 5]) * r);
+                            o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * r, __uint_as_float(v[8 * j + 7]) * r);
+                            *reinterpret_cast<uint4 *>(yrow + col) = o;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace gemm
+
+// ----------------------------------------------------------- host helpers
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][inner] (inner contiguous), box inner 64 x box_rows,
+// 128-byte swizzle; out-of-range elements of a box read as zero.
+qkn_status make_tmap(CUtensorMap *m, const void *ptr, int64_t rows, int64_t inner, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return fail(QKN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(inner * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)gemm::BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(QKN_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return QKN_OK;
+}
+
+qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float eps, cudaStream_t s) {
+    const int64_t blocks = (M + 7) / 8;
+    if (blocks > 0x7fffffffLL) return fail(QKN_ERR_SHAPE, "flashnorm_proj: M too large");
+    inv_rms_kernel<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), inv, M, K, eps);
+    return check_launch("inv_rms_kernel launch");
+}
+
+qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
+                       cudaStream_t s) {
+    CUtensorMap tx, tw;
+    if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
+    if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;
+    gemm::Args g;
+    g.inv_rms = inv;
+    g.y = static_cast<__nv_bfloat16 *>(y);
+    g.M = (int)M;
+    g.N = (int)N;
+    g.K = (int)K;
+    g.m_blocks = (int)((M + gemm::BM - 1) / gemm::BM);
+    g.n_blocks = (int)((N + gemm::BN - 1) / gemm::BN);
+    g.k_blocks = (int)((K + gemm::BK - 1) / gemm::BK);
+    g.num_tiles = g.m_blocks * g.n_blocks;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm::flashnorm_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             gemm::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(flashnorm_gemm_kernel)");
+        attr_set[dev] = true;
+    }
+    const int grid = g.num_tiles < sm_count() ? g.num_tiles : sm_count();
+    gemm::flashnorm_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tx, tw, g);
+    return check_launch("flashnorm_gemm_kernel launch");
+}
+
+}  // namespace
+}  // namespace qkn
+
+using namespace qkn;
+
+extern "C" QKN_API qkn_status flashnorm_fold_weights(const void *w, const void *W, void *W_folded, int64_t K,
+                                                     int64_t N, qkn_dtype wdt, int out_k_major, void *stream) {
+    if (!valid_dtype(wdt)) return fail(QKN_ERR_DTYPE, "flashnorm_fold_weights: unknown dtype %d", (int)wdt);
+    if (w == nullptr || W == nullptr || W_folded == nullptr)
+        return fail(QKN_ERR_NULL, "flashnorm_fold_weights: w, W and W_folded are required");
+    if (K < 0 || N < 0) return fail(QKN_ERR_SHAPE, "flashnorm_fold_weights: negative size");
+    if (!aligned(w, dtype_size(wdt)) || !aligned(W, 2) || !aligned(W_folded, 2))
+        return fail(QKN_ERR_ALIGN, "flashnorm_fold_weights: pointers must be aligned to their element size");
+    if (K == 0 || N == 0) return QKN_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const __nv_bfloat16 *Wb = static_cast<const __nv_bfloat16 *>(W);
+    __nv_bfloat16 *Wo = static_cast<__nv_bfloat16 *>(W_folded);
+    if (out_k_major) {
+        const int64_t gx = (N + kFoldTile - 1) / kFoldTile, gy = (K + kFoldTile - 1) / kFoldTile;
+        if (gx > 0x7fffffffLL || gy > 65535) return fail(QKN_ERR_SHAPE, "flashnorm_fold_weights: too large");
+        dim3 grid((unsigned)gx, (unsigned)gy);
+        if (wdt == QKN_BF16)
+            fold_transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(w), Wb, Wo, K, N);
+        else
+            fold_transpose_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float *>(w), Wb, Wo, K, N);
+    } else {
+        const int blocks = 4 * sm_count();
+        if (wdt == QKN_BF16)
+            fold_rowmajor_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(w), Wb, Wo, K, N);
+        else
+            fold_rowmajor_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float *>(w), Wb, Wo, K, N);
+    }
+    return check_launch("flashnorm_fold_weights launch");
+}
+
+extern "C" QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y, int64_t M, int64_t N,
+                                             int64_t K, int w_k_major, float eps, const float *inv_rms,
+                                             float *inv_rms_out, void *stream) {
+    if (x == nullptr || W_folded == nullptr || y == nullptr)
+        return fail(QKN_ERR_NULL, "flashnorm_proj: x, W_folded and y are required");
+    if (M < 1 || N < 1 || K < 1 || M > 0x7fffffffLL || N > 0x7fffffffLL || K > 0x7fffffffLL)
+        return fail(QKN_ERR_SHAPE, "flashnorm_proj: bad sizes M=%lld N=%lld K=%lld", (long long)M, (long long)N,
+                    (long long)K);
+    if (K % 8 != 0 || N % 8 != 0)
+        return fail(QKN_ERR_SHAPE, "flashnorm_proj: K=%lld and N=%lld must be multiples of 8", (long long)K,
+                    (long long)N);
+    if (!w_k_major) return fail(QKN_ERR_UNSUPPORTED, "flashnorm_proj: W_folded must be K-major ([N][K])");
+    if (inv_rms == nullptr && (!(eps >= 0.f) || isinf(eps)))
+        return fail(QKN_ERR_EPS, "flashnorm_proj: eps must be finite and >= 0");
+    if (!aligned(x, 16) || !aligned(W_folded, 16) || !aligned(y, 16) || (inv_rms && !aligned(inv_rms, 4)) ||
+        (inv_rms_out && !aligned(inv_rms_out, 4)))
+        return fail(QKN_ERR_ALIGN, "flashnorm_proj: x, W_folded and y must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float *inv = inv_rms;
+    float *scratch = nullptr;
+    if (inv == nullptr) {
+        float *dst = inv_rms_out;
+        if (dst == nullptr) {
+            cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&scratch), (size_t)M * sizeof(float), s);
+            if (e != cudaSuccess) return cuda_fail(e, "flashnorm_proj: cudaMallocAsync(inv_rms scratch)");
+            dst = scratch;
+        }
+        if (qkn_status st = launch_inv_rms(x, dst, M, K, eps, s)) {
+            if (scratch) cudaFreeAsync(scratch, s);
+            return st;
+        }
+        inv = dst;
+    }
+    qkn_status st = launch_gemm(x, W_folded, y, inv, M, N, K, s);
+    if (scratch) {
+        cudaError_t e = cudaFreeAsync(scratch, s);
+        if (st == QKN_OK && e != cudaSuccess) st = cuda_fail(e, "flashnorm_proj: cudaFreeAsync(inv_rms scratch)");
+    }
+    return st;
+}
+
+extern "C" QKN_API qkn_status qkn_check_device(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "qkn_check_device: stream synchronisation");
+    int flag = 0;
+    e = cudaMemcpyFromSymbol(&flag, g_device_error, sizeof flag);
+    if (e != cudaSuccess) return cuda_fail(e, "qkn_check_device: reading the device error word");
+    if (flag != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+        return fail(QKN_ERR_TIMEOUT, "a bounded device-side wait gave up (flag %d)", flag);
+    }
+    return QKN_OK;
+}

@@ -1,0 +1,91 @@
+"""Multi-process host logic on CPU: world size 2 over gloo.
+
+The GPU path needs no collective (tokens are independent); these tests cover
+what the ranks do share: seeding, row sharding, the max-over-ranks timing and
+the token accounting of the benchmark's value.
+"""
+from __future__ import annotations
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from rmsnorm_qknorm_b200 import dist as qdist
+from rmsnorm_qknorm_b200 import workloads as W
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # each rank's elapsed time differs; everyone must see the max
+        elapsed = 10.0 + 5.0 * rank
+        mx = qdist.max_over_ranks(elapsed)
+        tokens = qdist.sum_over_ranks(128.0)
+        # strong-scaling shards of one batch: disjoint, covering, reassembled in order
+        T = 1001
+        start, stop = qdist.shard_rows(T, rank, world)
+        inp = W.make_qknorm_inputs("prefill_gqa", seed=0, tokens=T, dq=64, dk=16)
+        mine = inp["q"][start:stop].float()
+        # reassemble the shards on every rank through padded buffers (shards differ by <= 1 row)
+        pad = (T + world - 1) // world
+        padded = torch.zeros(pad, 64)
+        padded[: stop - start] = mine
+        pbufs = [torch.empty(pad, 64) for _ in range(world)]
+        dist.all_gather(pbufs, padded)
+        spans = [qdist.shard_rows(T, r, world) for r in range(world)]
+        gathered = torch.cat([pb[: b - a] for pb, (a, b) in zip(pbufs, spans)])
+        # weak scaling: rank seeds give different batches, rank 0 keeps the workload seed
+        s0 = qdist.rank_seed(0, rank)
+        out[rank] = {
+            "max": mx, "tokens": tokens, "shard": (start, stop),
+            "reassembled_equal": bool(torch.equal(gathered, inp["q"].float())),
+            "seed": s0,
+        }
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gloo():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+        res = dict(out)
+    assert res[0]["max"] == res[1]["max"] == 15.0
+    assert res[0]["tokens"] == res[1]["tokens"] == 256.0
+    assert res[0]["shard"] == (0, 501) and res[1]["shard"] == (501, 1001)
+    assert res[0]["reassembled_equal"] and res[1]["reassembled_equal"]
+    assert res[0]["seed"] == 0 and res[1]["seed"] != 0
+
+
+@pytest.mark.parametrize("total,world", [(0, 1), (1, 4), (7, 3), (131072, 8), (16383, 8)])
+def test_shard_rows_partition(total, world):
+    spans = [qdist.shard_rows(total, r, world) for r in range(world)]
+    assert spans[0][0] == 0 and spans[-1][1] == total
+    for (a, b), (c, d) in zip(spans, spans[1:]):
+        assert b == c
+    sizes = [b - a for a, b in spans]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_shard_rows_rejects_bad_requests():
+    with pytest.raises(ValueError):
+        qdist.shard_rows(10, 2, 2)
+    with pytest.raises(ValueError):
+        qdist.shard_rows(10, 0, 0)
+
+
+def test_max_without_process_group_is_identity():
+    assert qdist.max_over_ranks(3.5) == 3.5

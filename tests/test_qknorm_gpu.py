@@ -1,0 +1,234 @@
+"""GPU parity of qknorm_fused and rmsnorm_partial_stats against the fp64 oracle.
+
+Every case calls the CUDA library through its C ABI (via the thin binding) and
+compares element by element with the oracle on the same inputs, copied back
+to the host exactly:
+
+* fp32 outputs: relative error <= 1e-5; bf16 outputs: within 1 bf16 ulp of the
+  oracle rounded once (round-to-nearest-even); partial sums: relative 1e-5.
+
+Sizes: every workload at oracle-friendly sizes that span several blocks with a
+ragged tail, the two small workloads at full size, and the two large ones at
+full size in the exact launch configuration the benchmark times, checked on
+sampled rows plus properties that hold for every row.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rmsnorm_qknorm_b200 as qk
+from parity import assert_bf16_close, assert_f32_close, PARTIAL_REL_TOL
+from rmsnorm_qknorm_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def check(out: torch.Tensor, x: torch.Tensor, w: torch.Tensor, eps: float, what: str):
+    ref = oracle.rmsnorm(x.cpu(), w.cpu(), eps)
+    if out.dtype == torch.bfloat16:
+        return assert_bf16_close(out, ref, what)
+    return assert_f32_close(out, ref, what=what)
+
+
+def run_pair(inp, **kw):
+    return qk.qknorm_fused(inp["q"], inp["k"], inp["wq"], inp["wk"], inp["eps"], inp["n_seg"], **kw)
+
+
+def to_dev(inp):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+# ------------------------------------------------------------- the four workloads
+
+
+@pytest.mark.parametrize("name,tokens", [("tiny", None), ("decode", None), ("prefill_gqa", 203),
+                                         ("long_context", 301)])
+def test_workload_parity_oracle_sized(cuda_lib, name, tokens):
+    inp = to_dev(W.make_qknorm_inputs(name, seed=0, tokens=tokens))
+    qo, ko = run_pair(inp)
+    torch.cuda.synchronize()
+    check(qo, inp["q"], inp["wq"], inp["eps"], f"{name} q")
+    check(ko, inp["k"], inp["wk"], inp["eps"], f"{name} k")
+
+
+def _full_size_sampled(name, n_sample=384):
+    wl = W.QKNORM_WORKLOADS[name]
+    inp = W.make_qknorm_inputs(name, seed=0, device=DEV)
+    qo, ko = run_pair(inp)
+    qo2, ko2 = run_pair(inp)
+    torch.cuda.synchronize()
+    # determinism: bitwise-equal outputs on a second call
+    assert torch.equal(qo.view(torch.int16), qo2.view(torch.int16))
+    assert torch.equal(ko.view(torch.int16), ko2.view(torch.int16))
+    g = torch.Generator().manual_seed(7)
+    rows = torch.unique(torch.cat([torch.tensor([0, 1, wl.tokens - 2, wl.tokens - 1]),
+                                   torch.randint(0, wl.tokens, (n_sample,), generator=g)]))
+    rd = rows.to(DEV)
+    check(qo[rd], inp["q"][rd], inp["wq"], wl.eps, f"{name} q sampled")
+    check(ko[rd], inp["k"][rd], inp["wk"], wl.eps, f"{name} k sampled")
+    # every row: finite, and (y / w) has unit mean square up to bf16 rounding
+    for y, w in ((qo, inp["wq"]), (ko, inp["wk"])):
+        z = y.float() / w.float()
+        ms = z.pow(2).mean(dim=1)
+        assert torch.isfinite(y.float()).all()
+        assert (ms - 1).abs().max().item() < 2e-2
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["prefill_gqa", "long_context"])
+def test_workload_parity_full_size(cuda_lib, name):
+    _full_size_sampled(name)
+
+
+# ------------------------------------------------------------------ n_seg coverage
+
+
+@pytest.mark.parametrize("n_seg", [1, 2, 4, 5, 8, 16, 64])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_n_seg(cuda_lib, n_seg, dtype):
+    T, d = 37, 1280  # 1280 = 2^8 * 5: every n_seg above divides it
+    g = torch.Generator().manual_seed(n_seg)
+    x = (torch.randn(T, d, generator=g) * 3).to(dtype).to(DEV)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(dtype).to(DEV)
+    y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, n_seg)
+    torch.cuda.synchronize()
+    check(y, x, w, 1e-6, f"n_seg={n_seg}")
+    p = qk.rmsnorm_partial_stats(x, n_seg)
+    torch.cuda.synchronize()
+    ref = oracle.segment_partials(x.cpu(), n_seg)
+    assert_f32_close(p, ref, tol=PARTIAL_REL_TOL, what=f"partials n_seg={n_seg}")
+
+
+# ------------------------------------------------------------- shapes and layouts
+
+
+@pytest.mark.parametrize("d", [1, 3, 8, 24, 100, 520, 1000, 4104, 65536, 65544, 131072])
+def test_widths(cuda_lib, d):
+    # odd widths and widths not a multiple of 8 take the element-wise kernel;
+    # 65536 bf16 is the widest row of the vector kernel, 131072 the element-wise one
+    T = 3 if d >= 65536 else 19
+    g = torch.Generator().manual_seed(d)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16).to(DEV)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16).to(DEV)
+    y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, 1)
+    torch.cuda.synchronize()
+    check(y, x, w, 1e-6, f"d={d}")
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 17, 255, 257, 1025])
+def test_ragged_token_counts(cuda_lib, T):
+    inp = to_dev(W.make_qknorm_inputs("prefill_gqa", seed=T, tokens=T))
+    qo, ko = run_pair(inp)
+    torch.cuda.synchronize()
+    check(qo, inp["q"], inp["wq"], inp["eps"], f"T={T} q")
+    check(ko, inp["k"], inp["wk"], inp["eps"], f"T={T} k")
+
+
+def test_empty(cuda_lib):
+    x = torch.empty(0, 128, dtype=torch.bfloat16, device=DEV)
+    w = torch.ones(128, dtype=torch.bfloat16, device=DEV)
+    y, _ = qk.qknorm_fused(x, x, w, w, 1e-6, 4)
+    assert y.shape == (0, 128)
+
+
+def test_fused_qkv_views_in_place(cuda_lib):
+    # q and k as strided views of one [T, dq + 2 dk] projection output, normalised in place
+    T, dq, dk = 96, 640, 128
+    g = torch.Generator().manual_seed(3)
+    qkv = torch.randn(T, dq + 2 * dk, generator=g).to(torch.bfloat16).to(DEV)
+    wq = (1 + 0.1 * torch.randn(dq, generator=g)).to(torch.bfloat16).to(DEV)
+    wk = (1 + 0.1 * torch.randn(dk, generator=g)).to(torch.bfloat16).to(DEV)
+    before = qkv.clone()
+    q, k = qkv[:, :dq], qkv[:, dq:dq + dk]
+    qk.qknorm_fused(q, k, wq, wk, 1e-6, 8, inplace=True)
+    torch.cuda.synchronize()
+    check(qkv[:, :dq], before[:, :dq], wq, 1e-6, "in-place q view")
+    check(qkv[:, dq:dq + dk], before[:, dq:dq + dk], wk, 1e-6, "in-place k view")
+    assert torch.equal(qkv[:, dq + dk:], before[:, dq + dk:])  # v untouched
+
+
+def test_strided_unaligned_pitch(cuda_lib):
+    # a pitch that breaks 16-byte row alignment takes the element-wise kernel
+    T, d = 33, 256
+    g = torch.Generator().manual_seed(5)
+    buf = torch.randn(T, d + 3, generator=g).to(torch.bfloat16).to(DEV)
+    x = buf[:, :d]
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16).to(DEV)
+    out = torch.empty(T, d + 5, dtype=torch.bfloat16, device=DEV)[:, :d]
+    y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, 4, q_out=out)
+    torch.cuda.synchronize()
+    assert y.data_ptr() == out.data_ptr()
+    check(y, x.contiguous(), w, 1e-6, "unaligned pitch")
+
+
+@pytest.mark.parametrize("act,wdt", [(torch.bfloat16, torch.float32), (torch.float32, torch.bfloat16)])
+def test_mixed_weight_dtype(cuda_lib, act, wdt):
+    T, d = 40, 2048
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(T, d, generator=g).to(act).to(DEV)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(wdt).to(DEV)
+    y, _ = qk.qknorm_fused(x, x, w, w, 1e-6, 4)
+    torch.cuda.synchronize()
+    check(y, x, w, 1e-6, f"act={act} w={wdt}")
+
+
+# -------------------------------------------------------------- degenerate values
+
+
+def test_zero_rows_and_special_values(cuda_lib):
+    d = 512
+    x = torch.randn(6, d).to(torch.bfloat16)
+    x[0] = 0.0                      # zero row, eps > 0 -> 0
+    x[1, 7] = float("inf")          # inf -> NaN/inf in that row only
+    x[2, 9] = float("nan")
+    x[3] = 1e-30                    # tiny: eps dominates
+    x[4] = 3e38                     # near bf16 max: the fp32 sum of squares overflows
+    w = torch.ones(d, dtype=torch.bfloat16)
+    xd, wd = x.to(DEV), w.to(DEV)
+    y, _ = qk.qknorm_fused(xd, None, wd, None, 1e-6, 1)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    assert torch.all(yc[0] == 0)
+    assert torch.isnan(yc[1]).sum() + torch.isinf(yc[1]).sum() > 0
+    assert torch.isnan(yc[2]).all()
+    # fp32 statistics: S = inf gives inv = 0, so the row comes out as zeros
+    # (the documented range limit of fp32 statistics; the fp64 oracle has none)
+    assert torch.all(yc[4] == 0)
+    ref3 = oracle.rmsnorm(x[3:4], w, 1e-6)
+    assert_bf16_close(y[3:4], ref3, "tiny row")
+    assert torch.equal(yc[5], yc[5])  # finite row untouched by neighbours
+    assert_bf16_close(y[5:6], oracle.rmsnorm(x[5:6], w, 1e-6), "row after special values")
+
+
+def test_zero_row_eps_zero_is_nan(cuda_lib):
+    x = torch.zeros(2, 64, dtype=torch.float32, device=DEV)
+    w = torch.ones(64, dtype=torch.float32, device=DEV)
+    y, _ = qk.qknorm_fused(x, None, w, None, 0.0, 2)
+    torch.cuda.synchronize()
+    assert torch.isnan(y).all()
+
+
+def test_scale_invariance_on_gpu(cuda_lib):
+    # RMSNorm(c x) = RMSNorm(x) for a power-of-two c (exact scaling, eps tiny)
+    x = torch.randn(64, 1024).to(torch.bfloat16).to(DEV)
+    w = (1 + 0.1 * torch.randn(1024)).to(torch.bfloat16).to(DEV)
+    a, _ = qk.qknorm_fused(x, None, w, None, 0.0, 8)
+    b, _ = qk.qknorm_fused(x * 64, None, w, None, 0.0, 8)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_partial_stats_full_size_rows(cuda_lib):
+    inp = W.make_qknorm_inputs("prefill_gqa", seed=0, device=DEV, tokens=4096)
+    for key in ("q", "k"):
+        p = qk.rmsnorm_partial_stats(inp[key], 8)
+        torch.cuda.synchronize()
+        ref = oracle.segment_partials(inp[key].cpu(), 8)
+        assert_f32_close(p, ref, tol=PARTIAL_REL_TOL, what=f"partials {key}")
+        # the combined statistic of the partials is the full-row statistic
+        full = oracle.segment_partials(inp[key].cpu(), 1)[:, 0]
+        np.testing.assert_allclose(oracle.combine_partials(p.cpu().double().numpy()), full, rtol=1e-5)

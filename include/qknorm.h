@@ -159,6 +159,37 @@ QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y,
                                   void *stream);
 
 /*
+ * flashnorm_proj_noalloc -- flashnorm_proj for callers that cannot allocate
+ * device memory during the call.
+ *
+ * No counterpart in the pages: FlashNorm describes the computation, not how
+ * its scratch is obtained.  This variant exists for callers that must not
+ * call cudaMalloc (or any allocator) at call time -- runtimes that plan the
+ * whole device memory up front and forbid allocations on the hot path,
+ * callers under a framework whose allocator owns the device, real-time loops
+ * that cannot absorb an allocator's latency.
+ *
+ * Same arguments and result as flashnorm_proj with inv_rms == inv_rms_out ==
+ * NULL: the 1/rms vector is computed from x and eps into a fixed 1 MiB array
+ * compiled into the library (a file-scope __device__ variable, present on
+ * every GPU that loads the library until the process exits) instead of into
+ * memory-pool scratch.  The call allocates nothing.
+ *
+ * Limits and caveats:
+ * - M <= 262144 rows; larger M returns QKN_ERR_SHAPE before any launch.
+ * - Every call on a GPU shares the one array: calls that overlap on the GPU
+ *   (e.g. on two streams at once) race on it and must be serialised by the
+ *   caller.  Each call writes the entries it reads, so the array's leftover
+ *   contents from an earlier call never reach the result.
+ * - The first call on a device (with that device current) looks up the
+ *   array's device address with cudaGetSymbolAddress and caches it; make that
+ *   first call before any stream capture.
+ */
+QKN_API qkn_status flashnorm_proj_noalloc(const void *x, const void *W_folded, void *y,
+                                          int64_t M, int64_t N, int64_t K, int w_k_major,
+                                          float eps, void *stream);
+
+/*
  * qkn_check_device -- synchronises `stream`, then reads and clears the
  * current device's error word.  Returns QKN_ERR_TIMEOUT when a bounded
  * device-side wait of an earlier launch (the projection kernel's mbarrier

@@ -12,6 +12,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "qkn_common.cuh"
 
 namespace qkn {
@@ -512,4 +514,81 @@ extern "C" QKN_API qkn_status qkn_check_device(void *stream) {
         return fail(QKN_ERR_TIMEOUT, "a bounded device-side wait gave up (flag %d)", flag);
     }
     return QKN_OK;
+}
+
+// ===================================================== no-allocation variant
+//
+// Some callers cannot allocate device memory at call time: serving runtimes
+// that plan every byte of the GPU up front and forbid allocations on the hot
+// path (so the footprint stays fixed and no allocator lock is taken), callers
+// running under a framework whose own allocator owns the whole device, and
+// real-time loops that cannot afford an allocator's latency spikes.  For them
+// flashnorm_proj_noalloc keeps the 1/rms vector in the fixed array below
+// instead of taking scratch from the CUDA memory pool.
+//
+// The array is a file-scope device variable: every GPU that loads this
+// library holds it (1 MiB) until the process exits, and every call on that
+// GPU shares it, so calls that overlap on the GPU race on it.  Each call
+// overwrites the entries it uses before reading them, so nothing has to start
+// at zero.  In host code the name g_noalloc_inv_rms is only a host-side
+// stand-in; its device address is fetched once per device with
+// cudaGetSymbolAddress (on the first call made with that device current) and
+// cached.
+
+namespace qkn {
+namespace {
+
+constexpr int64_t kNoAllocMaxRows = 262144;  // 1 MiB of fp32
+
+static __device__ __align__(256) float g_noalloc_inv_rms[kNoAllocMaxRows];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_inv_rms on the current device (set up once).
+qkn_status noalloc_scratch(float **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "flashnorm_proj_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(QKN_ERR_UNSUPPORTED, "flashnorm_proj_noalloc: device %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_inv_rms);
+        if (e != cudaSuccess || p == nullptr)
+            return cuda_fail(e, "flashnorm_proj_noalloc: cudaGetSymbolAddress(scratch)");
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return QKN_OK;
+}
+
+}  // namespace
+}  // namespace qkn
+
+extern "C" QKN_API qkn_status flashnorm_proj_noalloc(const void *x, const void *W_folded, void *y, int64_t M,
+                                                     int64_t N, int64_t K, int w_k_major, float eps,
+                                                     void *stream) {
+    if (x == nullptr || W_folded == nullptr || y == nullptr)
+        return fail(QKN_ERR_NULL, "flashnorm_proj_noalloc: x, W_folded and y are required");
+    if (M < 1 || N < 1 || K < 1 || N > 0x7fffffffLL || K > 0x7fffffffLL)
+        return fail(QKN_ERR_SHAPE, "flashnorm_proj_noalloc: bad sizes M=%lld N=%lld K=%lld", (long long)M,
+                    (long long)N, (long long)K);
+    if (M > kNoAllocMaxRows)
+        return fail(QKN_ERR_SHAPE,
+                    "flashnorm_proj_noalloc: M=%lld rows exceed the fixed scratch of %lld rows; split the "
+                    "call or use flashnorm_proj", (long long)M, (long long)kNoAllocMaxRows);
+    if (K % 8 != 0 || N % 8 != 0)
+        return fail(QKN_ERR_SHAPE, "flashnorm_proj_noalloc: K=%lld and N=%lld must be multiples of 8",
+                    (long long)K, (long long)N);
+    if (!w_k_major) return fail(QKN_ERR_UNSUPPORTED, "flashnorm_proj_noalloc: W_folded must be K-major ([N][K])");
+    if (!(eps >= 0.f) || isinf(eps)) return fail(QKN_ERR_EPS, "flashnorm_proj_noalloc: eps must be finite and >= 0");
+    if (!aligned(x, 16) || !aligned(W_folded, 16) || !aligned(y, 16))
+        return fail(QKN_ERR_ALIGN, "flashnorm_proj_noalloc: x, W_folded and y must be 16-byte aligned");
+    float *inv = nullptr;
+    if (qkn_status st = noalloc_scratch(&inv)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (qkn_status st = launch_inv_rms(x, inv, M, K, eps, s)) return st;
+    return launch_gemm(x, W_folded, y, inv, M, N, K, s);
 }

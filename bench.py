@@ -335,18 +335,38 @@ def run_qknorm(args, rank, world, local, pg):
 
     for i in range(max(args.warmup, 3)):
         step(i)
+    # Small batches run for a few microseconds, less than one host-side launch
+    # of the Python binding: capture them in a CUDA graph so the device time is
+    # measured, not the launch rate.  Large batches launch directly, with an
+    # event pair around every launch.
+    use_graph = per_set < 256 * 1024 * 1024
+    graph = None
+    if use_graph:
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(steps):
+                step(i)
+        graph.replay()
+        torch.cuda.synchronize()
     barrier(pg)
     clocks = ClockSampler() if rank == 0 else None
     if clocks:
         clocks.start()
         clocks.mark(True)
-    total_ms, launch_ms = time_launches(step, steps, stream)
+    if use_graph:
+        total_ms, _ = time_launches(lambda _i: graph.replay(), 1, torch.cuda.current_stream(dev))
+        launch_ms = [total_ms / steps]
+    else:
+        total_ms, launch_ms = time_launches(step, steps, stream)
     if clocks:
         clocks.mark(False)
     barrier(pg)
     total_ms = max_over_ranks(total_ms, pg)
     avg_launch_ms = max_over_ranks(statistics.mean(launch_ms), pg)
     clk = clocks.stop(gpu_index=local) if clocks else None
+    if graph is not None:
+        del graph
 
     ms_per_step = total_ms / steps
     value = global_tokens / (ms_per_step * 1e-3)
@@ -404,6 +424,8 @@ def run_qknorm(args, rank, world, local, pg):
                          "kernel": "rownorm_vec_kernel",
                          "algorithmic_bytes_per_launch": per_set,
                          "avg_launch_us": avg_launch_ms * 1e3,
+                         "launch_timing": ("CUDA graph of all timed steps; mean includes in-graph gaps"
+                                           if use_graph else "event pair around every launch"),
                          "peak_source": f"{pk_kind} HBM copy bandwidth",
                          "frac_of_8TBs": achieved / 8000.0},
             "cpu_baseline": cpu,

@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "qkn_common.cuh"
+#include "qkn_sync.cuh"
 
 namespace qkn {
 
@@ -98,7 +99,6 @@ constexpr int TMEM_COLS = 2 * ACC_COLS;                 // double-buffered accum
 constexpr int THREADS = 192;                            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;      // 2 s: far above any tile's latency
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -118,59 +118,6 @@ struct Args {
     int M, N, K;
     int m_blocks, n_blocks, k_blocks, num_tiles;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_timer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                 ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-// Waits for the phase with the given parity to complete.  Gives up after
-// kWaitTimeoutNs, records the failure in g_device_error and returns false.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer();
-    while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer() - t0 > kWaitTimeoutNs) {
-            atomicExch(&g_device_error, 1);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
-}
 
 // Shared-memory matrix descriptor for a K-major operand stored as rows of 64
 // bf16 (128 bytes) with the 128-byte swizzle: groups of 8 rows are 1024 bytes
@@ -236,7 +183,7 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             mbar_init(smem_u32(&acc_full[a]), 1);   // one tcgen05.commit
             mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrive per epilogue warp
         }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
     }
     if (warp == 1) {  // whole warp: allocate the two accumulators in tensor memory
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -256,7 +203,7 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
         for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
             const int m_blk = tile % g.m_blocks, n_blk = tile / g.m_blocks;
             for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u)) { ok = false; break; }
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &g_device_error)) { ok = false; break; }
                 if (lane == 0) {
                     const uint32_t fb = smem_u32(&full[stage]);
                     uint8_t *sa = smem + stage * STAGE_BYTES;
@@ -277,11 +224,11 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
         for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u)) break;
+            if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, &g_device_error)) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
             for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait(smem_u32(&full[stage]), phase)) { ok = false; break; }
+                if (!mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
@@ -309,7 +256,7 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             const int m_blk = tile % g.m_blocks, n_blk = tile / g.m_blocks;
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase)) break;
+            if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase, &g_device_error)) break;
             tc_fence_after();
             const int row = m_blk * BM + quarter * 32 + lane;
             const bool row_ok = row < g.M;
@@ -511,8 +458,11 @@ extern "C" QKN_API qkn_status qkn_check_device(void *stream) {
     if (flag != 0) {
         const int zero = 0;
         cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
-        return fail(QKN_ERR_TIMEOUT, "a bounded device-side wait gave up (flag %d)", flag);
     }
+    int norm_flag = 0;
+    if (qkn_status st = read_norm_error(&norm_flag)) return st;
+    if (flag != 0 || norm_flag != 0)
+        return fail(QKN_ERR_TIMEOUT, "a bounded device-side wait gave up (projection %d, norm %d)", flag, norm_flag);
     return QKN_OK;
 }
 

@@ -28,6 +28,9 @@ inline bool valid_dtype(int t) { return t == QKN_F32 || t == QKN_BF16; }
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Reads the norm kernels' device error word into *flag and clears it.
+qkn_status read_norm_error(int *flag);
+
 // ---------------------------------------------------------------- device side
 
 // Streaming 16-byte load: data read once, evict-first in L1 and L2.
@@ -125,6 +128,33 @@ template <>
 __device__ __forceinline__ void load_weights<__nv_bfloat16, 4>(const __nv_bfloat16 *w, float (&f)[4]) {
     uint2 a = ld_ro_v2(w);
     f[0] = bf16lo(a.x); f[1] = bf16hi(a.x); f[2] = bf16lo(a.y); f[3] = bf16hi(a.y);
+}
+
+// Same values as load_weights, through plain read-only-path intrinsics that
+// the compiler may batch and hoist (for kernels with registers to spare).
+template <typename TW, int E>
+__device__ __forceinline__ void load_weights_batched(const TW *w, float (&f)[E]) {
+    if constexpr (sizeof(TW) * E == 16) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(w));
+        if constexpr (E == 8) {
+            Chunk<__nv_bfloat16>::unpack(a, f);
+        } else {
+            Chunk<float>::unpack(a, f);
+        }
+    } else if constexpr (sizeof(TW) * E == 32) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(w));
+        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(w) + 1);
+        f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y); f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+        f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y); f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+    } else {
+        const uint2 a = __ldg(reinterpret_cast<const uint2 *>(w));
+        f[0] = bf16lo(a.x); f[1] = bf16hi(a.x); f[2] = bf16lo(a.y); f[3] = bf16hi(a.y);
+    }
+}
+
+// Streaming 16-byte store through the intrinsic (freely schedulable).
+__device__ __forceinline__ void st_stream_batched(void *p, uint4 v) {
+    __stcs(reinterpret_cast<uint4 *>(p), v);
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);

@@ -15,8 +15,12 @@
 #include <math.h>
 
 #include "qkn_common.cuh"
+#include "qkn_sync.cuh"
 
 namespace qkn {
+
+// Set by a bounded wait of the staged kernel that gave up (see qkn_check_device).
+__device__ int g_norm_error = 0;
 
 constexpr int kFastMaxSeg = 8;    // segments handled by the vectorised kernel
 constexpr int kMaxWarps = 32;     // 1024-thread blocks at most
@@ -184,6 +188,405 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) rownorm_vec_kernel(const 
 }
 
 // ---------------------------------------------------------------------------
+// Staged kernel (rows up to ~40 KiB): persistent, one block per SM.
+//
+// Rows reach shared memory through 1-D bulk copies (cp.async.bulk, completion
+// counted on an mbarrier per stage), so the loads in flight do not depend on
+// what the threads are computing.  Every warp is both producer and consumer:
+// warp w handles every W-th "tile" of the block (whole rows of one job, at
+// most one stage of bytes) and owns `spw` stages of its own; as soon as it has
+// read a stage it refills it with its tile spw steps ahead, so while it works
+// on one stage the copies into its other stages are in flight, and no warp
+// ever waits for another warp's progress.  A warp reads each row twice from
+// shared memory -- the segment statistic, then the apply -- and writes the
+// output from registers with streaming stores.  The weights of both jobs are
+// widened to fp32 once per block and kept in shared memory, split into the
+// low and high 16-byte halves of each chunk so a warp's weight loads are
+// conflict-free.  Products use the packed fp32x2 pipe (two fp32 lanes per
+// instruction, each rounded exactly like a scalar fp32 operation).
+//
+// Segment partials: a lane's chunks c = lane, lane + 32, ... visit segments
+// in increasing order, so the lane keeps one running (even, odd) pair of sums
+// and parks their total in a per-warp shared-memory slot [segment][lane] when
+// it crosses a segment boundary.  The eight slots are then reduced over the
+// warp by recursive halving (lane bit 4 splits segments 0-3 / 4-7, bit 3 and
+// bit 2 split further, bits 1 and 0 finish the sum), after which lanes
+// 4j .. 4j+3 hold segment j; the segments are combined left to right.
+namespace staged {
+
+#ifndef QKN_STAGED_SMEM_LIMIT
+#define QKN_STAGED_SMEM_LIMIT (227 * 1024)
+#endif
+#ifndef QKN_STAGED_MAX_WARPS
+#define QKN_STAGED_MAX_WARPS 8
+#endif
+#ifndef QKN_STAGED_MAX_SPW
+#define QKN_STAGED_MAX_SPW 3
+#endif
+
+constexpr int kSmemLimit = QKN_STAGED_SMEM_LIMIT;    // whole dynamic shared memory
+constexpr int kMaxWarps = QKN_STAGED_MAX_WARPS;       // consumer warps
+constexpr int kMaxStagesPerWarp = QKN_STAGED_MAX_SPW;
+constexpr int kMaxThreads = 32 * kMaxWarps;
+#ifndef QKN_STAGED_UNROLL
+#define QKN_STAGED_UNROLL 4
+#endif
+constexpr int kUnroll = QKN_STAGED_UNROLL;             // chunks per lane per group
+static_assert(kFastMaxSeg == 8, "the warp reduction below is written for 8 segment slots");
+
+struct Job {
+    const uint8_t *x;
+    uint8_t *y;
+    const void *w;
+    int64_t ld_bytes, ldo_bytes, rows;
+    int d, row_bytes, nchunks, seg_chunks;
+    int w_offset;        // byte offset of this job's fp32 weights in shared memory
+    int rows_per_tile;
+    int64_t ntiles;
+};
+
+struct Args {
+    Job job[2];
+    int njobs;
+    int64_t total_tiles;
+    int n_seg;
+    float eps;
+    float *partial;
+    int warps;        // consumer warps W
+    int stages;       // W * stages per warp
+    int stage_bytes;  // multiple of 16
+    int w_bytes;      // fp32 weights of both jobs
+};
+
+// Shared memory: [ring][fp32 weights][full bars][W x 8 x 32 floats]
+inline int smem_bytes(int warps, int stages, int stage_bytes, int w_bytes) {
+    return stages * stage_bytes + w_bytes + stages * 8 + warps * kFastMaxSeg * 32 * 4;
+}
+
+__device__ __forceinline__ Job pick(const Args &a, int which) {
+    const Job &j0 = a.job[0], &j1 = a.job[1];
+    Job J;
+    J.x = which ? j1.x : j0.x;
+    J.y = which ? j1.y : j0.y;
+    J.w = which ? j1.w : j0.w;
+    J.ld_bytes = which ? j1.ld_bytes : j0.ld_bytes;
+    J.ldo_bytes = which ? j1.ldo_bytes : j0.ldo_bytes;
+    J.rows = which ? j1.rows : j0.rows;
+    J.d = which ? j1.d : j0.d;
+    J.row_bytes = which ? j1.row_bytes : j0.row_bytes;
+    J.nchunks = which ? j1.nchunks : j0.nchunks;
+    J.seg_chunks = which ? j1.seg_chunks : j0.seg_chunks;
+    J.w_offset = which ? j1.w_offset : j0.w_offset;
+    J.rows_per_tile = which ? j1.rows_per_tile : j0.rows_per_tile;
+    J.ntiles = which ? j1.ntiles : j0.ntiles;
+    return J;
+}
+
+// fp32 pairs of a 16-byte activation chunk.
+template <typename TA> struct Pairs;
+template <> struct Pairs<__nv_bfloat16> {
+    static constexpr int P = 4;
+    __device__ __forceinline__ static void get(const uint4 &v, float2 (&p)[P]) {
+        p[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+        p[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+        p[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+        p[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
+    }
+    __device__ __forceinline__ static uint4 put(const float2 (&p)[P]) {
+        return make_uint4(pack_bf16x2(p[0].x, p[0].y), pack_bf16x2(p[1].x, p[1].y),
+                          pack_bf16x2(p[2].x, p[2].y), pack_bf16x2(p[3].x, p[3].y));
+    }
+};
+template <> struct Pairs<float> {
+    static constexpr int P = 2;
+    __device__ __forceinline__ static void get(const uint4 &v, float2 (&p)[P]) {
+        p[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+        p[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+    }
+    __device__ __forceinline__ static uint4 put(const float2 (&p)[P]) {
+        return make_uint4(__float_as_uint(p[0].x), __float_as_uint(p[0].y), __float_as_uint(p[1].x),
+                          __float_as_uint(p[1].y));
+    }
+};
+
+// Sum of squares of one 16-byte chunk as an (even, odd) pair: a short
+// dependency chain per chunk, so the chunks of a group overlap.
+template <typename TA>
+__device__ __forceinline__ float2 chunk_sumsq(const uint4 &v) {
+    float2 p[Pairs<TA>::P];
+    Pairs<TA>::get(v, p);
+    float2 a = __fmul2_rn(p[0], p[0]);
+#pragma unroll
+    for (int i = 1; i < Pairs<TA>::P; ++i) a = __ffma2_rn(p[i], p[i], a);
+    return a;
+}
+
+// Adds a chunk's sum into the running pair sum, parking the running sum of
+// the segment being left whenever chunk c crosses a segment boundary.
+__device__ __forceinline__ void accumulate(float2 sq, int c, float2 &cur, int &cur_seg, int &next_bound,
+                                           int seg_chunks, float *part, int lane) {
+    while (c >= next_bound) {
+        part[cur_seg * 32 + lane] = cur.x + cur.y;
+        cur = make_float2(0.f, 0.f);
+        ++cur_seg;
+        next_bound += seg_chunks;
+    }
+    cur = __fadd2_rn(cur, sq);
+}
+
+// y = (x * inv) * w for one chunk c, stored with a streaming store.
+template <typename TA>
+__device__ __forceinline__ void apply_chunk(const uint4 &v, int c, float2 inv2, const float4 *wsm, int nchunks,
+                                            uint8_t *yr) {
+    float4 w[Pairs<TA>::P / 2];
+#pragma unroll
+    for (int h = 0; h < Pairs<TA>::P / 2; ++h) w[h] = wsm[h * nchunks + c];
+    float2 p[Pairs<TA>::P];
+    Pairs<TA>::get(v, p);
+#pragma unroll
+    for (int h = 0; h < Pairs<TA>::P / 2; ++h) {
+        p[2 * h] = __fmul2_rn(__fmul2_rn(p[2 * h], inv2), make_float2(w[h].x, w[h].y));
+        p[2 * h + 1] = __fmul2_rn(__fmul2_rn(p[2 * h + 1], inv2), make_float2(w[h].z, w[h].w));
+    }
+    st_stream_batched(yr + (int64_t)c * 16, Pairs<TA>::put(p));
+}
+
+// One row held in shared memory, processed by one warp.  `part` is the warp's
+// [8][32] scratch for lane partials; `wsm` the job's fp32 weights.
+template <typename TA, bool STATS>
+__device__ __forceinline__ void process_row(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
+                                            int64_t row, int lane, float *part) {
+    const int nchunks = J.nchunks;
+    const int n_seg = a.n_seg;
+    const int sc = J.seg_chunks;
+
+    // ---- statistic
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
+    float2 cur = make_float2(0.f, 0.f);
+    int cur_seg = 0, next_bound = sc;
+    int c0 = 0;
+    constexpr int G = 32 * kUnroll;  // chunks per group
+    if (nchunks >= G) {
+        // groups of kUnroll chunks per lane; the next group's loads are issued
+        // before the current group's arithmetic
+        uint4 vn[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) vn[u] = *reinterpret_cast<const uint4 *>(srow + (u * 32 + lane) * 16);
+        for (; c0 + G <= nchunks; c0 += G) {
+            uint4 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) v[u] = vn[u];
+            if (c0 + 2 * G <= nchunks) {
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    vn[u] = *reinterpret_cast<const uint4 *>(srow + (c0 + G + u * 32 + lane) * 16);
+            }
+            float2 sq[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) sq[u] = chunk_sumsq<TA>(v[u]);
+            if (c0 + (kUnroll - 1) * 32 + lane < next_bound) {  // the whole group is in the current segment
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) cur = __fadd2_rn(cur, sq[u]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    accumulate(sq[u], c0 + u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
+            }
+        }
+    }
+    for (; c0 < nchunks; c0 += 32) {
+        const int c = c0 + lane;
+        if (c < nchunks)
+            accumulate(chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)), c, cur, cur_seg,
+                       next_bound, sc, part, lane);
+    }
+    part[cur_seg * 32 + lane] = cur.x + cur.y;
+    __syncwarp();
+
+    float S = 0.f;
+    if (n_seg == 1) {
+        float r = part[lane];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+        S = r;
+        if constexpr (STATS) {
+            if (lane == 0) a.partial[row] = r;
+        }
+    } else {
+        float v8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v8[j] = part[j * 32 + lane];
+        const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+        float k4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float give = b4 ? v8[i] : v8[i + 4];
+            k4[i] = (b4 ? v8[i + 4] : v8[i]) + __shfl_xor_sync(0xffffffffu, give, 16);
+        }
+        float k2[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float give = b3 ? k4[i] : k4[i + 2];
+            k2[i] = (b3 ? k4[i + 2] : k4[i]) + __shfl_xor_sync(0xffffffffu, give, 8);
+        }
+        float r = (b2 ? k2[1] : k2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? k2[0] : k2[1], 4);
+        r += __shfl_xor_sync(0xffffffffu, r, 2);
+        r += __shfl_xor_sync(0xffffffffu, r, 1);
+        // lanes 4j .. 4j+3 now hold segment j; combine left to right
+        for (int j = 0; j < n_seg; ++j) S += __shfl_sync(0xffffffffu, r, 4 * j);
+        if constexpr (STATS) {
+            if ((lane & 3) == 0 && (lane >> 2) < n_seg) a.partial[row * n_seg + (lane >> 2)] = r;
+        }
+    }
+    __syncwarp();  // the scratch is rewritten by the next row
+
+    // ---- apply
+    if constexpr (!STATS) {
+        const float inv = rsqrtf(S / (float)J.d + a.eps);
+        const float2 inv2 = make_float2(inv, inv);
+        uint8_t *yr = J.y + row * J.ldo_bytes;
+        int c1 = 0;
+        if (nchunks >= G) {
+            uint4 vn[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) vn[u] = *reinterpret_cast<const uint4 *>(srow + (u * 32 + lane) * 16);
+            for (; c1 + G <= nchunks; c1 += G) {
+                uint4 v[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) v[u] = vn[u];
+                if (c1 + 2 * G <= nchunks) {
+#pragma unroll
+                    for (int u = 0; u < kUnroll; ++u)
+                        vn[u] = *reinterpret_cast<const uint4 *>(srow + (c1 + G + u * 32 + lane) * 16);
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) apply_chunk<TA>(v[u], c1 + u * 32 + lane, inv2, wsm, nchunks, yr);
+            }
+        }
+        for (; c1 < nchunks; c1 += 32) {
+            const int c = c1 + lane;
+            if (c < nchunks) apply_chunk<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16), c, inv2, wsm, nchunks, yr);
+        }
+    }
+}
+
+// Issues the bulk copies of one tile into a stage (one lane).
+__device__ __forceinline__ void issue_tile(const Args &a, int64_t tile, int64_t nt0, uint8_t *stage_ptr,
+                                           uint64_t *bar) {
+    const int which = tile >= nt0 ? 1 : 0;
+    const Job J = pick(a, which);
+    const int64_t row0 = (tile - (which ? nt0 : 0)) * J.rows_per_tile;
+    const int64_t left = J.rows - row0;
+    const int nrows = left < J.rows_per_tile ? (int)left : J.rows_per_tile;
+    const uint32_t fb = smem_u32(bar);
+    mbar_arrive_expect_tx(fb, (uint32_t)(nrows * J.row_bytes));
+    const uint32_t dst = smem_u32(stage_ptr);
+    for (int r = 0; r < nrows; ++r)
+        bulk_g2s(dst + r * J.row_bytes, J.x + (row0 + r) * J.ld_bytes, (uint32_t)J.row_bytes, fb);
+}
+
+template <typename TA, typename TW, bool STATS>
+__global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Args a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int W = a.warps, SB = a.stage_bytes;
+    const int spw = a.stages / W;
+    uint8_t *wbase = smem + (size_t)a.stages * SB;
+    uint64_t *full = reinterpret_cast<uint64_t *>(wbase + a.w_bytes);
+    float *scratch = reinterpret_cast<float *>(full + a.stages);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.stages; ++s) mbar_init(smem_u32(&full[s]), 1);  // issuing lane + bytes
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    // Warp w handles this block's tiles w, w + W, w + 2W, ... (k-th: w + k W)
+    // and owns stages w*spw .. w*spw + spw - 1; tile k lives in stage
+    // w*spw + k % spw.  The warp refills a stage itself as soon as it has
+    // read it, so no other warp's progress delays its copies.
+    const int64_t nt0 = a.job[0].ntiles;
+    const int64_t step = (int64_t)W * gridDim.x;
+    const int64_t first = blockIdx.x + (int64_t)warp * gridDim.x;
+    float *part = scratch + warp * kFastMaxSeg * 32;
+    int64_t issued = 0;  // tiles of this warp whose copies were issued
+    if (lane == 0) {
+        for (int j = 0; j < spw; ++j) {
+            const int64_t tile = first + j * step;
+            if (tile >= a.total_tiles) break;
+            issue_tile(a, tile, nt0, smem + (size_t)(warp * spw + j) * SB, &full[warp * spw + j]);
+            ++issued;
+        }
+    }
+    issued = __shfl_sync(0xffffffffu, issued, 0);
+
+    if constexpr (!STATS) {
+        // while the first tiles are in flight: the weights of both jobs,
+        // widened to fp32, chunk halves de-interleaved; loads batched 4 deep
+        constexpr int E = Chunk<TA>::E;
+        for (int i = 0; i < a.njobs; ++i) {
+            const Job J = pick(a, i);
+            const TW *w = static_cast<const TW *>(J.w);
+            float *dst = reinterpret_cast<float *>(wbase + J.w_offset);
+            for (int c0 = 0; c0 < J.nchunks; c0 += 4 * (int)blockDim.x) {
+                float f[4][E];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * (int)blockDim.x + (int)threadIdx.x;
+                    if (c < J.nchunks) load_weights_batched<TW, E>(w + (int64_t)c * E, f[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * (int)blockDim.x + (int)threadIdx.x;
+                    if (c < J.nchunks) {
+#pragma unroll
+                        for (int h = 0; h < E / 4; ++h)
+                            reinterpret_cast<float4 *>(dst)[h * J.nchunks + c] =
+                                make_float4(f[u][4 * h], f[u][4 * h + 1], f[u][4 * h + 2], f[u][4 * h + 3]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    int64_t k = 0;
+    for (int64_t tile = first; tile < a.total_tiles; tile += step, ++k) {
+        const int slot = (int)(k % spw);
+        const int stage = warp * spw + slot;
+        const uint32_t par = (uint32_t)(k / spw) & 1u;
+        if (!mbar_wait(smem_u32(&full[stage]), par, &g_norm_error)) break;
+        const int which = tile >= nt0 ? 1 : 0;
+        const Job J = pick(a, which);
+        const int64_t row0 = (tile - (which ? nt0 : 0)) * J.rows_per_tile;
+        const int64_t left = J.rows - row0;
+        const int nrows = left < J.rows_per_tile ? (int)left : J.rows_per_tile;
+        const uint8_t *sbase = smem + (size_t)stage * SB;
+        const float4 *wsm = reinterpret_cast<const float4 *>(wbase + J.w_offset);
+        for (int r = 0; r < nrows; ++r)
+            process_row<TA, STATS>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
+        __syncwarp();
+        // refill this stage with the warp's tile k + spw
+        const int64_t next = tile + spw * step;
+        if (next < a.total_tiles) {
+            if (lane == 0) {
+                // the generic-proxy reads of this stage precede the async-proxy writes
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                issue_tile(a, next, nt0, smem + (size_t)stage * SB, &full[stage]);
+            }
+            ++issued;
+        }
+    }
+    // drain: copies this warp issued but did not consume (only after a failed
+    // wait) must land before the block exits
+    for (; k < issued; ++k)
+        mbar_wait(smem_u32(&full[warp * spw + (int)(k % spw)]), (uint32_t)(k / spw) & 1u, &g_norm_error);
+}
+
+}  // namespace staged
+
+// ---------------------------------------------------------------------------
 // Element-wise kernel for any alignment, width and n_seg <= QKN_MAX_SEG: one
 // row per 256-thread block; each segment is reduced over the block in turn.
 // The row is read a second time (from L2) for the apply step.
@@ -264,6 +667,74 @@ qkn_status launch_vec(RowArgs &a, int njobs, cudaStream_t s) {
     return check_launch("rownorm_vec_kernel launch");
 }
 
+// Ring geometry for the staged kernel: stage = the widest row (rounded up to
+// 16 bytes); as many consumer warps (at most kMaxWarps) as allow two stages
+// per warp next to the fp32 weights within the shared-memory limit.  Returns
+// false when even 2 warps x 2 stages do not fit (the register kernel runs).
+bool staged_geometry(int64_t max_row_bytes, int64_t w_bytes, int *warps, int *spw, int *stage_bytes) {
+    const int64_t sb = (max_row_bytes + 15) / 16 * 16;
+    for (int w = staged::kMaxWarps; w >= 2; --w) {
+        const int64_t fixed = w_bytes + w * kFastMaxSeg * 32 * 4 + 8 * w * staged::kMaxStagesPerWarp;
+        int64_t per_warp = (staged::kSmemLimit - fixed) / (w * sb);
+        if (per_warp > staged::kMaxStagesPerWarp) per_warp = staged::kMaxStagesPerWarp;
+        if (per_warp >= 2) {
+            *warps = w;
+            *spw = (int)per_warp;
+            *stage_bytes = (int)sb;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <typename TA, typename TW, bool STATS>
+qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps, float *partial,
+                         int warps, int spw, int stage_bytes, cudaStream_t s) {
+    constexpr int E = Chunk<TA>::E;
+    staged::Args a{};
+    a.njobs = njobs;
+    a.n_seg = n_seg;
+    a.eps = eps;
+    a.partial = partial;
+    a.total_tiles = 0;
+    a.warps = warps;
+    a.stages = warps * spw;
+    a.stage_bytes = stage_bytes;
+    a.w_bytes = 0;
+    for (int i = 0; i < njobs; ++i) {
+        const Tensor2 &t = ts[i];
+        staged::Job &J = a.job[i];
+        J.x = static_cast<const uint8_t *>(t.x);
+        J.y = static_cast<uint8_t *>(t.y);
+        J.w = t.w;
+        J.ld_bytes = t.ld * (int64_t)sizeof(TA);
+        J.ldo_bytes = t.ldo * (int64_t)sizeof(TA);
+        J.rows = rows;
+        J.d = (int)t.d;
+        J.row_bytes = (int)(t.d * (int64_t)sizeof(TA));
+        J.nchunks = (int)(t.d / E);
+        J.seg_chunks = J.nchunks / n_seg;
+        J.w_offset = a.w_bytes;
+        if (!STATS) a.w_bytes += (int)(t.d * 4);
+        J.rows_per_tile = stage_bytes / J.row_bytes;
+        J.ntiles = (rows + J.rows_per_tile - 1) / J.rows_per_tile;
+        a.total_tiles += J.ntiles;
+    }
+    const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes);
+    static int attr_bytes[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || attr_bytes[dev] < smem) {
+        cudaError_t e = cudaFuncSetAttribute(staged::rownorm_staged_kernel<TA, TW, STATS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rownorm_staged_kernel)");
+        if (dev >= 0 && dev < 64) attr_bytes[dev] = smem;
+    }
+    const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
+    staged::rownorm_staged_kernel<TA, TW, STATS><<<(unsigned)grid, 32 * a.warps, smem, s>>>(a);
+    return check_launch("rownorm_staged_kernel launch");
+}
+
 template <typename TA, typename TW, bool STATS>
 qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps,
                     float *partial, cudaStream_t s) {
@@ -293,6 +764,17 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
             if (max_chunks <= (int64_t)kVecCfgs[c].cpt * kVecCfgs[c].block) { cfg = c; break; }
         }
         if (cfg < 0) vec = false;
+    }
+
+    if (vec) {
+        int64_t max_row_bytes = 0;
+        for (int i = 0; i < njobs; ++i)
+            if (ts[i].d * (int64_t)sizeof(TA) > max_row_bytes) max_row_bytes = ts[i].d * (int64_t)sizeof(TA);
+        int64_t w_bytes = 0;
+        for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
+        int warps = 0, spw = 0, sb = 0;
+        if (staged_geometry(max_row_bytes, w_bytes, &warps, &spw, &sb))
+            return launch_staged<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, warps, spw, sb, s);
     }
 
     if (vec) {
@@ -418,3 +900,16 @@ extern "C" QKN_API qkn_status rmsnorm_partial_stats(const void *x, int64_t rows,
     return dispatch_types<true>(act, act, &t, 1, rows, n_seg, 0.f, partial,
                                 static_cast<cudaStream_t>(stream));
 }
+
+namespace qkn {
+// Reads and clears the staged kernel's device error word (current device).
+qkn_status read_norm_error(int *flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_norm_error, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the norm kernel's device error word");
+    if (*flag) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_norm_error, &zero, sizeof zero);
+    }
+    return QKN_OK;
+}
+}  // namespace qkn

@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--strong", action="store_true",
                     help="split one batch over the ranks (strong scaling) instead of one batch per rank")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the QK-Norm workload's tokens per GPU (smaller cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline work budget")
     return ap.parse_args()
@@ -315,11 +317,12 @@ def run_qknorm(args, rank, world, local, pg):
     steps = args.steps if args.steps is not None else (2000 if wl.tokens >= 100000 else 5000)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
+    batch = wl.tokens if args.tokens is None else args.tokens
     if args.strong:
-        r0, r1 = qdist.shard_rows(wl.tokens, rank, world)
-        my_tokens, global_tokens = r1 - r0, wl.tokens
+        r0, r1 = qdist.shard_rows(batch, rank, world)
+        my_tokens, global_tokens = r1 - r0, batch
     else:
-        my_tokens, global_tokens = wl.tokens, world * wl.tokens
+        my_tokens, global_tokens = batch, world * batch
     per_set = wl.algorithmic_bytes(my_tokens)
     nsets = 1 if per_set > 2 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_set))
     sets = []
@@ -372,8 +375,9 @@ def run_qknorm(args, rank, world, local, pg):
     value = global_tokens / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
     achieved = per_set / (avg_launch_ms * 1e-3) / 1e9
-    src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh"]
-    traffic = traffic_for("rownorm_vec_kernel", wl.name, src)
+    src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
+           "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
+    traffic = traffic_for("rownorm_staged_kernel", wl.name, src) if args.tokens is None else None
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -421,7 +425,7 @@ def run_qknorm(args, rank, world, local, pg):
                               f"{nsets} rotating input sets totalling {nsets * per_set / 1e6:.0f} MB > L2")},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                         "kernel": "rownorm_vec_kernel",
+                         "kernel": "rownorm_staged_kernel",
                          "algorithmic_bytes_per_launch": per_set,
                          "avg_launch_us": avg_launch_ms * 1e3,
                          "launch_timing": ("CUDA graph of all timed steps; mean includes in-graph gaps"
@@ -488,7 +492,8 @@ def run_flashnorm(args, rank, world, local, pg):
     value = world * wl.M / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
     tflops = wl.flops() / (avg_gemm * 1e-3) / 1e12
-    src = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh"]
+    src = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
+           "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
 
     e2e = None
     if args.e2e_steps > 0:

@@ -146,12 +146,16 @@ QKN_API qkn_status flashnorm_fold_weights(const void *w, const void *W, void *W_
  * W_folded   [N][K] bf16 (K contiguous, out_k_major == 1 of the fold);
  *            w_k_major must be 1 (0 returns QKN_ERR_UNSUPPORTED)
  * y          [M][N] bf16, row-major
- * inv_rms    optional [M] fp32 precomputed 1/rms; NULL = compute from x and eps
- * inv_rms_out optional [M] fp32 that receives the 1/rms used (when inv_rms is
- *            NULL); when both are NULL the library takes stream-ordered
- *            scratch of M floats from the CUDA memory pool for the call
+ * inv_rms    optional [M] fp32 precomputed 1/rms (then used as given)
+ * inv_rms_out optional [M] fp32; when inv_rms is NULL and this is given, a
+ *            row-statistics pass writes each row's 1/rms here and the
+ *            projection reads it (the faster form: the matmul keeps all of
+ *            shared-memory bandwidth)
+ * With both NULL the projection kernel computes each row's 1/rms itself from
+ * the x tiles it streams for the matmul, in parallel with the tensor-core
+ * work -- no extra pass and no workspace.
  * Sizes: M, N, K >= 1; K and N multiples of 8.  Pointers 16-byte aligned.
- * y must not overlap x or W_folded.
+ * y must not overlap x or W_folded.  Nothing is allocated.
  */
 QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y,
                                   int64_t M, int64_t N, int64_t K, int w_k_major,
@@ -170,10 +174,11 @@ QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y,
  * that cannot absorb an allocator's latency.
  *
  * Same arguments and result as flashnorm_proj with inv_rms == inv_rms_out ==
- * NULL: the 1/rms vector is computed from x and eps into a fixed 1 MiB array
- * compiled into the library (a file-scope __device__ variable, present on
- * every GPU that loads the library until the process exits) instead of into
- * memory-pool scratch.  The call allocates nothing.
+ * NULL (equal up to the summation order of the row statistic): a row-
+ * statistics pass writes the 1/rms vector into a fixed 1 MiB array compiled
+ * into the library (a file-scope __device__ variable, present on every GPU
+ * that loads the library until the process exits), then the projection reads
+ * it.  The call allocates nothing.
  *
  * Limits and caveats:
  * - M <= 262144 rows; larger M returns QKN_ERR_SHAPE before any launch.

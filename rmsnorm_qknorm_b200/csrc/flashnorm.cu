@@ -63,23 +63,40 @@ __global__ void __launch_bounds__(256) fold_transpose_kernel(const TW *__restric
 
 // ======================================================= row statistics
 
-// inv[m] = 1/sqrt(sum_k x[m][k]^2 / K + eps), one warp per row, 16-byte loads.
-// K is a multiple of 8 and rows are 16-byte aligned (checked by the caller).
+// inv[m] = 1/sqrt(sum_k x[m][k]^2 / K + eps), one warp per row, 16-byte loads
+// issued 8 deep per lane before any arithmetic (a 4096-wide row is then one
+// round trip).  K is a multiple of 8 and rows are 16-byte aligned (checked by
+// the caller).
 __global__ void __launch_bounds__(256) inv_rms_kernel(const __nv_bfloat16 *__restrict__ x,
                                                       float *__restrict__ inv, int64_t M, int64_t K,
                                                       float eps) {
+    constexpr int U = 8;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= M) return;  // whole warp leaves together
     const uint8_t *xr = reinterpret_cast<const uint8_t *>(x + row * K);
     const int64_t nchunks = K / 8;
-    float s = 0.f;
-    for (int64_t c = lane; c < nchunks; c += 32) {
-        float f[8];
-        Chunk<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4 *>(xr + c * 16)), f);
+    float2 s2 = make_float2(0.f, 0.f);
+    for (int64_t c0 = 0; c0 < nchunks; c0 += 32 * U) {
+        uint4 v[U];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s = fmaf(f[e], f[e], s);
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = c0 + u * 32 + lane;
+            v[u] = c < nchunks ? __ldcs(reinterpret_cast<const uint4 *>(xr + c * 16)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float2 p0 = make_float2(bf16lo(v[u].x), bf16hi(v[u].x));
+            const float2 p1 = make_float2(bf16lo(v[u].y), bf16hi(v[u].y));
+            const float2 p2 = make_float2(bf16lo(v[u].z), bf16hi(v[u].z));
+            const float2 p3 = make_float2(bf16lo(v[u].w), bf16hi(v[u].w));
+            s2 = __ffma2_rn(p0, p0, s2);
+            s2 = __ffma2_rn(p1, p1, s2);
+            s2 = __ffma2_rn(p2, p2, s2);
+            s2 = __ffma2_rn(p3, p3, s2);
+        }
     }
+    float s = s2.x + s2.y;
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (lane == 0) inv[row] = rsqrtf(s / (float)K + eps);
 }
@@ -96,9 +113,11 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int UMMA_K = 16;                              // K of one kind::f16 MMA
 constexpr int ACC_COLS = BN;                            // fp32 accumulator: one column per n
 constexpr int TMEM_COLS = 2 * ACC_COLS;                 // double-buffered accumulator
-constexpr int THREADS = 192;                            // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-7 row statistics
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
+constexpr int INV_BYTES = 2 * BM * 4;                   // 1/rms of the rows of both accumulator tiles
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + INV_BYTES + 1024;  // + 1 KiB for alignment
+constexpr int GROUP_M = 16;  // tiles are walked in groups of 16 row blocks so concurrent tiles share operands in L2
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -113,11 +132,27 @@ constexpr uint32_t kInstrDesc = (1u << 4)                 // D format: f32
                               | ((uint32_t)(BM >> 4) << 24);
 
 struct Args {
-    const float *inv_rms;   // [M]
+    const float *inv_rms;   // [M] given 1/rms (used when compute_inv == 0)
+    float *inv_out;         // [M] optional: receives the 1/rms computed in-kernel
     __nv_bfloat16 *y;       // [M][N]
     int M, N, K;
     int m_blocks, n_blocks, k_blocks, num_tiles;
+    int compute_inv;        // 1: rows' 1/rms from the x tiles streaming through shared memory
+    float eps;
 };
+
+// Tile index -> (row block, column block), walking GROUP_M row blocks at a
+// time down each column block: the ~148 tiles in flight at once then touch
+// at most GROUP_M x-blocks and a handful of W'-blocks.
+__device__ __forceinline__ void tile_coords(int tile, const Args &g, int &m_blk, int &n_blk) {
+    const int group_tiles = GROUP_M * g.n_blocks;
+    const int group = tile / group_tiles;
+    const int first_m = group * GROUP_M;
+    const int rows_in_group = min(g.m_blocks - first_m, GROUP_M);
+    const int in_group = tile - group * group_tiles;
+    m_blk = first_m + in_group % rows_in_group;
+    n_blk = in_group / rows_in_group;
+}
 
 // Shared-memory matrix descriptor for a K-major operand stored as rows of 64
 // bf16 (128 bytes) with the 128-byte swizzle: groups of 8 rows are 1024 bytes
@@ -170,18 +205,22 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+    uint64_t *stats_full = bars + 2 * STAGES + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 6);
+    float *inv_buf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);  // [2][BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 1);    // producer's arrive + TMA bytes
-            mbar_init(smem_u32(&empty[s]), 1);   // one tcgen05.commit
+            // one tcgen05.commit, plus one arrive per statistics warp when they read x
+            mbar_init(smem_u32(&empty[s]), g.compute_inv ? 3 : 1);
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(smem_u32(&acc_full[a]), 1);   // one tcgen05.commit
-            mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrive per epilogue warp
+            mbar_init(smem_u32(&acc_full[a]), 1);    // one tcgen05.commit
+            mbar_init(smem_u32(&acc_empty[a]), 4);   // one arrive per epilogue warp
+            mbar_init(smem_u32(&stats_full[a]), 2);  // one arrive per statistics warp
         }
         mbar_init_fence();
     }
@@ -201,7 +240,8 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
         uint32_t phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
-            const int m_blk = tile % g.m_blocks, n_blk = tile / g.m_blocks;
+            int m_blk, n_blk;
+            tile_coords(tile, g, m_blk, n_blk);
             for (int kb = 0; kb < g.k_blocks; ++kb) {
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &g_device_error)) { ok = false; break; }
                 if (lane == 0) {
@@ -248,19 +288,26 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             if (lane == 0) umma_commit(smem_u32(&acc_full[acc]));  // accumulator ready
             __syncwarp();
         }
-    } else {
+    } else if (warp < 6) {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
         const int quarter = warp & 3;  // TMEM lanes this warp may access: 32 * quarter ...
         int it = 0;
         for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++it) {
-            const int m_blk = tile % g.m_blocks, n_blk = tile / g.m_blocks;
+            int m_blk, n_blk;
+            tile_coords(tile, g, m_blk, n_blk);
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase, &g_device_error)) break;
             tc_fence_after();
             const int row = m_blk * BM + quarter * 32 + lane;
             const bool row_ok = row < g.M;
-            const float r = row_ok ? __ldg(g.inv_rms + row) : 0.f;
+            float r;
+            if (g.compute_inv) {
+                if (!mbar_wait(smem_u32(&stats_full[acc]), acc_phase, &g_device_error)) break;
+                r = inv_buf[acc * BM + quarter * 32 + lane];
+            } else {
+                r = row_ok ? __ldg(g.inv_rms + row) : 0.f;
+            }
             __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll 1
@@ -286,6 +333,65 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+        }
+    } else if (g.compute_inv) {
+        // ---------------------------------------------------------------- row statistics (warps 6, 7)
+        // FlashNorm's RMS runs beside the matmul: each x tile the TMA brings in
+        // for the MMA is also read here, and every row's sum of squares over K
+        // accumulates while the tensor cores work.  The 128-byte swizzle only
+        // permutes the 16-byte chunks inside a row, so a row's chunks are read
+        // in logical order j at physical position j ^ (row & 7).  Lane l of
+        // statistics warp sw owns rows sw*64 + l and sw*64 + l + 32.
+        const int sw = warp - 6;
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x, ++it) {
+            int m_blk, n_blk;
+            tile_coords(tile, g, m_blk, n_blk);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            float2 ssq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            for (int kb = 0; kb < g.k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
+                const uint8_t *a_tile = smem + stage * STAGE_BYTES;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int r = sw * 64 + lane + 32 * i;
+                    const uint8_t *arow = a_tile + r * (BK * 2);
+                    uint4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4 *>(arow + ((j ^ (r & 7)) * 16));
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float2 p0 = make_float2(bf16lo(v[j].x), bf16hi(v[j].x));
+                        const float2 p1 = make_float2(bf16lo(v[j].y), bf16hi(v[j].y));
+                        const float2 p2 = make_float2(bf16lo(v[j].z), bf16hi(v[j].z));
+                        const float2 p3 = make_float2(bf16lo(v[j].w), bf16hi(v[j].w));
+                        ssq[i] = __ffma2_rn(p0, p0, ssq[i]);
+                        ssq[i] = __ffma2_rn(p1, p1, ssq[i]);
+                        ssq[i] = __ffma2_rn(p2, p2, ssq[i]);
+                        ssq[i] = __ffma2_rn(p3, p3, ssq[i]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[stage]));
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            // inv_buf[acc] is free once the epilogue has finished tile it - 2
+            if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, &g_device_error)) break;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = sw * 64 + lane + 32 * i;
+                const float inv = rsqrtf((ssq[i].x + ssq[i].y) / (float)g.K + g.eps);
+                inv_buf[acc * BM + r] = inv;
+                const int row = m_blk * BM + r;
+                if (g.inv_out != nullptr && n_blk == 0 && row < g.M) g.inv_out[row] = inv;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&stats_full[acc]));
         }
     }
 
@@ -344,13 +450,18 @@ qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float
     return check_launch("inv_rms_kernel launch");
 }
 
+// inv == nullptr: the kernel computes every row's 1/rms itself (eps) and,
+// when inv_out is given, stores it there.
 qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t s) {
+                       float eps, float *inv_out, cudaStream_t s) {
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;
     gemm::Args g;
     g.inv_rms = inv;
+    g.inv_out = inv_out;
+    g.compute_inv = inv == nullptr ? 1 : 0;
+    g.eps = eps;
     g.y = static_cast<__nv_bfloat16 *>(y);
     g.M = (int)M;
     g.N = (int)N;
@@ -426,27 +537,14 @@ extern "C" QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded
         (inv_rms_out && !aligned(inv_rms_out, 4)))
         return fail(QKN_ERR_ALIGN, "flashnorm_proj: x, W_folded and y must be 16-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const float *inv = inv_rms;
-    float *scratch = nullptr;
-    if (inv == nullptr) {
-        float *dst = inv_rms_out;
-        if (dst == nullptr) {
-            cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&scratch), (size_t)M * sizeof(float), s);
-            if (e != cudaSuccess) return cuda_fail(e, "flashnorm_proj: cudaMallocAsync(inv_rms scratch)");
-            dst = scratch;
-        }
-        if (qkn_status st = launch_inv_rms(x, dst, M, K, eps, s)) {
-            if (scratch) cudaFreeAsync(scratch, s);
-            return st;
-        }
-        inv = dst;
+    if (inv_rms == nullptr && inv_rms_out != nullptr) {
+        // the caller's buffer is the workspace of a separate row-statistics
+        // pass, which leaves the matmul's shared-memory bandwidth to the MMA
+        if (qkn_status st = launch_inv_rms(x, inv_rms_out, M, K, eps, s)) return st;
+        inv_rms = inv_rms_out;
     }
-    qkn_status st = launch_gemm(x, W_folded, y, inv, M, N, K, s);
-    if (scratch) {
-        cudaError_t e = cudaFreeAsync(scratch, s);
-        if (st == QKN_OK && e != cudaSuccess) st = cuda_fail(e, "flashnorm_proj: cudaFreeAsync(inv_rms scratch)");
-    }
-    return st;
+    // with no 1/rms at all the GEMM computes it beside the matmul (no workspace)
+    return launch_gemm(x, W_folded, y, inv_rms, M, N, K, eps, nullptr, s);
 }
 
 extern "C" QKN_API qkn_status qkn_check_device(void *stream) {
@@ -540,5 +638,5 @@ extern "C" QKN_API qkn_status flashnorm_proj_noalloc(const void *x, const void *
     if (qkn_status st = noalloc_scratch(&inv)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (qkn_status st = launch_inv_rms(x, inv, M, K, eps, s)) return st;
-    return launch_gemm(x, W_folded, y, inv, M, N, K, s);
+    return launch_gemm(x, W_folded, y, inv, M, N, K, eps, nullptr, s);
 }

@@ -258,7 +258,7 @@ struct Args {
     int w_bytes;      // fp32 weights of both jobs
 };
 
-// Shared memory: [ring][fp32 weights][full bars][W x 8 x 32 floats]
+// Shared memory: [ring][fp32 weights][full bars][W x 8 x 32 floats scratch]
 inline int smem_bytes(int warps, int stages, int stage_bytes, int w_bytes) {
     return stages * stage_bytes + w_bytes + stages * 8 + warps * kFastMaxSeg * 32 * 4;
 }
@@ -502,10 +502,33 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
     }
     __syncthreads();
 
+    // The first batch of weight loads goes out before the tile copies, so it
+    // does not queue behind them in the memory system; the weights are
+    // widened and stored while the copies stream in.
+    constexpr int E = Chunk<TA>::E;
+    constexpr int WB = 4;  // weight chunks per thread per batch
+    float wf[2][WB][E];
+    if constexpr (!STATS) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (i < a.njobs) {
+                const Job J = pick(a, i);
+                const TW *w = static_cast<const TW *>(J.w);
+#pragma unroll
+                for (int u = 0; u < WB; ++u) {
+                    const int c = u * (int)blockDim.x + (int)threadIdx.x;
+                    if (c < J.nchunks) load_weights_batched<TW, E>(w + (int64_t)c * E, wf[i][u]);
+                }
+            }
+        }
+    }
+
     // Warp w handles this block's tiles w, w + W, w + 2W, ... (k-th: w + k W)
     // and owns stages w*spw .. w*spw + spw - 1; tile k lives in stage
     // w*spw + k % spw.  The warp refills a stage itself as soon as it has
-    // read it, so no other warp's progress delays its copies.
+    // read it, so no other warp's progress delays its copies.  (Claiming
+    // tiles dynamically from a block-wide counter measured slower: the fixed
+    // dealing keeps the whole grid streaming through memory in order.)
     const int64_t nt0 = a.job[0].ntiles;
     const int64_t step = (int64_t)W * gridDim.x;
     const int64_t first = blockIdx.x + (int64_t)warp * gridDim.x;
@@ -522,27 +545,34 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
     issued = __shfl_sync(0xffffffffu, issued, 0);
 
     if constexpr (!STATS) {
-        // while the first tiles are in flight: the weights of both jobs,
-        // widened to fp32, chunk halves de-interleaved; loads batched 4 deep
-        constexpr int E = Chunk<TA>::E;
-        for (int i = 0; i < a.njobs; ++i) {
+        // weights of both jobs as fp32 in shared memory, chunk halves de-interleaved
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (i >= a.njobs) break;
             const Job J = pick(a, i);
             const TW *w = static_cast<const TW *>(J.w);
-            float *dst = reinterpret_cast<float *>(wbase + J.w_offset);
-            for (int c0 = 0; c0 < J.nchunks; c0 += 4 * (int)blockDim.x) {
-                float f[4][E];
+            float4 *dst = reinterpret_cast<float4 *>(wbase + J.w_offset);
+            for (int c0 = 0; c0 < J.nchunks; c0 += WB * (int)blockDim.x) {
+                float f[WB][E];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < WB; ++u) {
                     const int c = c0 + u * (int)blockDim.x + (int)threadIdx.x;
-                    if (c < J.nchunks) load_weights_batched<TW, E>(w + (int64_t)c * E, f[u]);
+                    if (c < J.nchunks) {
+                        if (c0 == 0) {
+#pragma unroll
+                            for (int e = 0; e < E; ++e) f[u][e] = wf[i][u][e];  // loaded above
+                        } else {
+                            load_weights_batched<TW, E>(w + (int64_t)c * E, f[u]);
+                        }
+                    }
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < WB; ++u) {
                     const int c = c0 + u * (int)blockDim.x + (int)threadIdx.x;
                     if (c < J.nchunks) {
 #pragma unroll
                         for (int h = 0; h < E / 4; ++h)
-                            reinterpret_cast<float4 *>(dst)[h * J.nchunks + c] =
+                            dst[h * J.nchunks + c] =
                                 make_float4(f[u][4 * h], f[u][4 * h + 1], f[u][4 * h + 2], f[u][4 * h + 3]);
                     }
                 }

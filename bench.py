@@ -338,20 +338,18 @@ def run_qknorm(args, rank, world, local, pg):
 
     for i in range(max(args.warmup, 3)):
         step(i)
-    # Small batches run for a few microseconds, less than one host-side launch
-    # of the Python binding: capture them in a CUDA graph so the device time is
-    # measured, not the launch rate.  Large batches launch directly, with an
-    # event pair around every launch.
-    use_graph = per_set < 256 * 1024 * 1024
-    graph = None
-    if use_graph:
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for i in range(steps):
-                step(i)
-        graph.replay()
-        torch.cuda.synchronize()
+    # The timed launches are captured in one CUDA graph and replayed: the
+    # device time of back-to-back launches is measured, not the Python
+    # binding's launch rate or the per-launch front-end latency (small batches
+    # run for a few microseconds, less than one host-side launch).
+    use_graph = True
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(steps):
+            step(i)
+    graph.replay()
+    torch.cuda.synchronize()
     barrier(pg)
     clocks = ClockSampler() if rank == 0 else None
     if clocks:
@@ -428,8 +426,8 @@ def run_qknorm(args, rank, world, local, pg):
                          "kernel": "rownorm_staged_kernel",
                          "algorithmic_bytes_per_launch": per_set,
                          "avg_launch_us": avg_launch_ms * 1e3,
-                         "launch_timing": ("CUDA graph of all timed steps; mean includes in-graph gaps"
-                                           if use_graph else "event pair around every launch"),
+                         "launch_timing": "one CUDA graph of all timed launches, CUDA events around its "
+                                          "replay; the mean includes the in-graph gaps between launches",
                          "peak_source": f"{pk_kind} HBM copy bandwidth",
                          "frac_of_8TBs": achieved / 8000.0},
             "cpu_baseline": cpu,

@@ -114,6 +114,33 @@ QKN_API qkn_status rmsnorm_partial_stats(const void *x, int64_t rows, int64_t d,
                                          float *partial, void *stream);
 
 /*
+ * rmsnorm_apply_partials -- the apply step of tensor-parallel QK-Norm.
+ *
+ * Defined by: SwiftQK, abstract -- under tensor parallelism each shard holds
+ * a slice of the row and only the shards' scalar sums of squares are
+ * exchanged; every shard then normalises its own slice with the combined
+ * statistic.  With the n_part partials of each row gathered (for example
+ * rmsnorm_partial_stats on every shard plus an all-gather of the scalars):
+ *   S      = ((p_0 + p_1) + p_2) + ... + p_{n_part-1}   (fixed order, fp32)
+ *   y[r][i] = (x[r][i] * rsqrt(S / d_full + eps)) * w[i]
+ *
+ * x, y     [rows][d] this shard's slice, pitches ld, ld_out (y may equal x)
+ * w        [d] this shard's slice of the weights
+ * partial  fp32; the j-th partial of row r is
+ *          partial[r * part_row_stride + j * part_stride]
+ *          (rmsnorm_partial_stats output: strides n_seg, 1; an all-gathered
+ *          [n_part][rows] array: strides 1, rows)
+ * n_part   1 .. 4096;  d_full = width of the whole row (the mean's divisor),
+ *          d <= d_full <= 2^24
+ */
+QKN_API qkn_status rmsnorm_apply_partials(const void *x, const void *w, void *y,
+                                          int64_t rows, int64_t d, int64_t ld, int64_t ld_out,
+                                          const float *partial, int n_part,
+                                          int64_t part_row_stride, int64_t part_stride,
+                                          int64_t d_full, qkn_dtype act, qkn_dtype wdt,
+                                          float eps, void *stream);
+
+/*
  * flashnorm_fold_weights -- fold the RMSNorm weights into the next linear
  * layer (offline).
  *
@@ -161,6 +188,32 @@ QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y,
                                   int64_t M, int64_t N, int64_t K, int w_k_major,
                                   float eps, const float *inv_rms, float *inv_rms_out,
                                   void *stream);
+
+/*
+ * qkv_norm_proj -- QKV projection with QKV-normalisation, pre-attention
+ * RMSNorm eliminated.
+ *
+ * Defined by: FlashNorm, abstract -- by the scale invariance of RMS, an
+ * RMSNorm followed by a linear layer followed by another RMSNorm allows the
+ * first RMSNorm to be eliminated (models that normalise q, k and v).  With
+ * the pre-attention norm's weights folded into W' (flashnorm_fold_weights),
+ * its 1/rms(x) cancels in the per-row norms that follow:
+ *   u       = x W'^T                         (no row scaling; bf16 out)
+ *   y[:, 0:nq)          = RMSNorm(u_q; wq, eps)   with n_seg partials
+ *   y[:, nq:nq+nk)      = RMSNorm(u_k; wk, eps)
+ *   y[:, nq+nk:nq+nk+nv) = RMSNorm(u_v; wv, eps)  (when nv > 0)
+ * Exact up to rounding when the eliminated norm's eps is 0; with eps > 0 the
+ * two differ by the relative size of that eps next to the rows' mean square.
+ *
+ * x [M][K] bf16; W_folded [nq+nk+nv][K] bf16 (K contiguous); y [M][nq+nk+nv]
+ * bf16; wq, wk, wv weights of dtype wdt.  K and nq+nk+nv multiples of 8;
+ * nq, nk, nv multiples of n_seg; x, W_folded, y 16-byte aligned.  Three
+ * launches (projection, q+k norm, v norm) on `stream`; nothing is allocated.
+ */
+QKN_API qkn_status qkv_norm_proj(const void *x, const void *W_folded, void *y,
+                                 int64_t M, int64_t K, int64_t nq, int64_t nk, int64_t nv,
+                                 const void *wq, const void *wk, const void *wv,
+                                 qkn_dtype wdt, float eps, int n_seg, void *stream);
 
 /*
  * flashnorm_proj_noalloc -- flashnorm_proj for callers that cannot allocate

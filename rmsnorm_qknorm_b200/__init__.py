@@ -15,6 +15,10 @@ Entry points (same names as the C ABI):
 * :func:`flashnorm_fold_weights` -- FlashNorm's W' = diag(w) W.
 * :func:`flashnorm_proj` -- y = (x W') * 1/rms(x), the deferred-normalisation
   GEMM with the scaling in the epilogue.
+* :func:`rmsnorm_apply_partials` -- the apply step of tensor-parallel QK-Norm:
+  normalise a shard from the gathered per-shard partial sums.
+* :func:`qkv_norm_proj` -- QKV projection + QKV-normalisation with the
+  pre-attention RMSNorm eliminated (FlashNorm's scale-invariance identity).
 """
 from __future__ import annotations
 
@@ -32,6 +36,8 @@ __all__ = [
     "rmsnorm_partial_stats",
     "flashnorm_fold_weights",
     "flashnorm_proj",
+    "rmsnorm_apply_partials",
+    "qkv_norm_proj",
     "STATUS_NAMES",
     "QKN_MAX_SEG",
 ]
@@ -79,8 +85,12 @@ def load_library() -> ctypes.CDLL:
         lib.rmsnorm_partial_stats.argtypes = [p, i64, i64, i64, i32, i32, p, p]
         lib.flashnorm_fold_weights.argtypes = [p, p, p, i64, i64, i32, i32, p]
         lib.flashnorm_proj.argtypes = [p, p, p, i64, i64, i64, i32, f32, p, p, p]
+        lib.rmsnorm_apply_partials.argtypes = [p, p, p, i64, i64, i64, i64, p, i32, i64, i64, i64,
+                                               i32, i32, f32, p]
+        lib.qkv_norm_proj.argtypes = [p, p, p, i64, i64, i64, i64, i64, p, p, p, i32, f32, i32, p]
+        lib.qkn_check_device.argtypes = [p]
         for f in ("qknorm_fused", "rmsnorm_partial_stats", "flashnorm_fold_weights",
-                  "flashnorm_proj"):
+                  "flashnorm_proj", "rmsnorm_apply_partials", "qkv_norm_proj", "qkn_check_device"):
             getattr(lib, f).restype = ctypes.c_int
         lib.qkn_last_error.restype = ctypes.c_char_p
         lib.qkn_last_error.argtypes = []
@@ -245,4 +255,64 @@ def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *
         inv_rms.data_ptr() if inv_rms is not None else None,
         inv_rms_out.data_ptr() if inv_rms_out is not None else None, _stream(stream))
     _check("flashnorm_proj", st)
+    return out
+
+
+def rmsnorm_apply_partials(x: torch.Tensor, w: torch.Tensor, partial: torch.Tensor, d_full: int,
+                           eps: float = 1e-6, *, out: torch.Tensor | None = None,
+                           inplace: bool = False, stream=None) -> torch.Tensor:
+    """Normalise the shard x [rows, d] given every row's partial sums of squares.
+
+    ``partial`` is fp32 and 2-D: [rows, n_part] (e.g. rmsnorm_partial_stats
+    output) or [n_part, rows] (e.g. an all-gather of per-shard partials); the
+    layout is read from its strides and its first dimension's length.
+    ``d_full`` is the width of the whole row the partials cover.
+    """
+    rows, d, ld = _rows(x, "x")
+    act = _dtype_code(x.dtype)
+    _vec(w, "w", d)
+    _cuda(partial, "partial")
+    if partial.dtype != torch.float32 or partial.dim() != 2:
+        raise ValueError("partial must be a 2-D fp32 tensor")
+    if partial.shape[0] == rows:
+        n_part, prs, ps = partial.shape[1], partial.stride(0), partial.stride(1)
+    elif partial.shape[1] == rows:
+        n_part, prs, ps = partial.shape[0], partial.stride(1), partial.stride(0)
+    else:
+        raise ValueError(f"partial {tuple(partial.shape)} does not match {rows} rows")
+    if inplace:
+        y, ldo = x, ld
+    else:
+        y = out if out is not None else torch.empty((rows, d), dtype=x.dtype, device=x.device)
+        _, _, ldo = _rows(y, "out")
+    st = load_library().rmsnorm_apply_partials(
+        x.data_ptr(), w.data_ptr(), y.data_ptr(), rows, d, ld, ldo, partial.data_ptr(), int(n_part),
+        int(prs), int(ps), int(d_full), act, _dtype_code(w.dtype), float(eps), _stream(stream))
+    _check("rmsnorm_apply_partials", st)
+    return y
+
+
+def qkv_norm_proj(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, nv: int,
+                  wq: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor | None, eps: float = 1e-6,
+                  n_seg: int = 1, *, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """[q | k | v] = per-group RMSNorm of x W_folded^T; the pre-attention RMSNorm eliminated."""
+    _cuda(x, "x")
+    _cuda(W_folded, "W_folded")
+    if x.dim() != 2 or not x.is_contiguous() or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a contiguous bf16 [M, K] tensor")
+    M, K = x.shape
+    N = nq + nk + nv
+    if tuple(W_folded.shape) != (N, K) or not W_folded.is_contiguous() or W_folded.dtype != torch.bfloat16:
+        raise ValueError(f"W_folded must be a contiguous bf16 [{N}, {K}] tensor")
+    _vec(wq, "wq", nq)
+    _vec(wk, "wk", nk)
+    if nv > 0:
+        _vec(wv, "wv", nv)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    st = load_library().qkv_norm_proj(
+        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, K, nq, nk, nv, wq.data_ptr(),
+        wk.data_ptr(), wv.data_ptr() if (wv is not None and nv > 0) else None, _dtype_code(wq.dtype),
+        float(eps), int(n_seg), _stream(stream))
+    _check("qkv_norm_proj", st)
     return out

@@ -138,6 +138,7 @@ struct Args {
     int M, N, K;
     int m_blocks, n_blocks, k_blocks, num_tiles;
     int compute_inv;        // 1: rows' 1/rms from the x tiles streaming through shared memory
+    int unit_scale;         // 1: no row scaling at all (y = x W'^T)
     float eps;
 };
 
@@ -302,7 +303,9 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             const int row = m_blk * BM + quarter * 32 + lane;
             const bool row_ok = row < g.M;
             float r;
-            if (g.compute_inv) {
+            if (g.unit_scale) {
+                r = 1.f;
+            } else if (g.compute_inv) {
                 if (!mbar_wait(smem_u32(&stats_full[acc]), acc_phase, &g_device_error)) break;
                 r = inv_buf[acc * BM + quarter * 32 + lane];
             } else {
@@ -453,14 +456,15 @@ qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float
 // inv == nullptr: the kernel computes every row's 1/rms itself (eps) and,
 // when inv_out is given, stores it there.
 qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
-                       float eps, float *inv_out, cudaStream_t s) {
+                       float eps, float *inv_out, cudaStream_t s, bool unit_scale = false) {
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;
     gemm::Args g;
     g.inv_rms = inv;
     g.inv_out = inv_out;
-    g.compute_inv = inv == nullptr ? 1 : 0;
+    g.unit_scale = unit_scale ? 1 : 0;
+    g.compute_inv = (inv == nullptr && !unit_scale) ? 1 : 0;
     g.eps = eps;
     g.y = static_cast<__nv_bfloat16 *>(y);
     g.M = (int)M;
@@ -639,4 +643,45 @@ extern "C" QKN_API qkn_status flashnorm_proj_noalloc(const void *x, const void *
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (qkn_status st = launch_inv_rms(x, inv, M, K, eps, s)) return st;
     return launch_gemm(x, W_folded, y, inv, M, N, K, eps, nullptr, s);
+}
+
+// ===================================================== RMSNorm elimination
+//
+// FlashNorm, abstract: by the scale invariance of RMS, RMSNorm -> linear ->
+// RMSNorm lets the first RMSNorm be dropped.  With q, k and v each
+// RMS-normalised after the projection (QKV-normalisation), the pre-attention
+// RMSNorm reduces to its weights, already folded into W', and its 1/rms(x)
+// disappears: per row, RMSNorm(c * u) = RMSNorm(u) for the scale c = 1/rms(x)
+// (exactly when that norm's eps is 0; otherwise up to the relative size of
+// eps next to the rows' mean square).  So: y = x W'^T with no row scaling,
+// then the q / k / v row groups normalised in place.
+extern "C" QKN_API qkn_status qkv_norm_proj(const void *x, const void *W_folded, void *y, int64_t M, int64_t K,
+                                            int64_t nq, int64_t nk, int64_t nv, const void *wq, const void *wk,
+                                            const void *wv, qkn_dtype wdt, float eps, int n_seg, void *stream) {
+    if (!valid_dtype(wdt)) return fail(QKN_ERR_DTYPE, "qkv_norm_proj: unknown dtype %d", (int)wdt);
+    if (x == nullptr || W_folded == nullptr || y == nullptr || wq == nullptr || wk == nullptr ||
+        (nv > 0 && wv == nullptr))
+        return fail(QKN_ERR_NULL, "qkv_norm_proj: x, W_folded, y, wq, wk (and wv when nv > 0) are required");
+    const int64_t N = nq + nk + nv;
+    if (M < 1 || K < 1 || nq < 1 || nk < 1 || nv < 0 || M > 0x7fffffffLL || N > 0x7fffffffLL || K > 0x7fffffffLL)
+        return fail(QKN_ERR_SHAPE, "qkv_norm_proj: bad sizes M=%lld K=%lld nq=%lld nk=%lld nv=%lld", (long long)M,
+                    (long long)K, (long long)nq, (long long)nk, (long long)nv);
+    if (K % 8 != 0 || N % 8 != 0)
+        return fail(QKN_ERR_SHAPE, "qkv_norm_proj: K and nq + nk + nv must be multiples of 8");
+    if (n_seg < 1 || n_seg > QKN_MAX_SEG || nq % n_seg || nk % n_seg || nv % n_seg)
+        return fail(QKN_ERR_SHAPE, "qkv_norm_proj: nq, nk, nv must be multiples of n_seg=%d", n_seg);
+    if (!(eps >= 0.f) || isinf(eps)) return fail(QKN_ERR_EPS, "qkv_norm_proj: eps must be finite and >= 0");
+    if (!aligned(x, 16) || !aligned(W_folded, 16) || !aligned(y, 16))
+        return fail(QKN_ERR_ALIGN, "qkv_norm_proj: x, W_folded and y must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (qkn_status st = launch_gemm(x, W_folded, y, nullptr, M, N, K, 0.f, nullptr, s, /*unit_scale=*/true))
+        return st;
+    __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(y);
+    if (qkn_status st = qknorm_fused(yb, yb + nq, wq, wk, nullptr, nullptr, M, nq, nk, N, N, N, N, QKN_BF16, wdt,
+                                     eps, n_seg, stream))
+        return st;
+    if (nv > 0)
+        return qknorm_fused(yb + nq + nk, nullptr, wv, nullptr, nullptr, nullptr, M, nv, 0, N, 0, N, 0, QKN_BF16,
+                            wdt, eps, n_seg, stream);
+    return QKN_OK;
 }

@@ -137,3 +137,27 @@ def test_binding_rejects_cpu_tensors():
     w = torch.ones(64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         qk.qknorm_fused(x, None, w, None)
+
+
+def test_apply_partials_validation(lib):
+    f = lib.rmsnorm_apply_partials
+    # (x, w, y, rows, d, ld, ld_out, partial, n_part, prs, ps, d_full, act, wdt, eps, stream)
+    assert f(None, P, P, 4, 64, 64, 64, P, 8, 8, 1, 512, BF16, BF16, 1e-6, None) == NULL
+    assert f(P, P, P, 4, 64, 32, 64, P, 8, 8, 1, 512, BF16, BF16, 1e-6, None) == SHAPE  # ld < d
+    assert f(P, P, P, 4, 64, 64, 64, P, 8, 8, 1, 32, BF16, BF16, 1e-6, None) == SHAPE   # d_full < d
+    assert f(P, P, P, 4, 64, 64, 64, P, 0, 8, 1, 512, BF16, BF16, 1e-6, None) == SHAPE  # n_part
+    assert f(P, P, P, 4, 64, 64, 64, P, 8, 8, 1, 512, 9, BF16, 1e-6, None) == DTYPE
+    assert f(P, P, P, 4, 64, 64, 64, P, 8, 8, 1, 512, BF16, BF16, -1.0, None) == EPS
+    assert f(P, P, P, 4, 64, 64, 64, P + 2, 8, 8, 1, 512, BF16, BF16, 1e-6, None) == ALIGN
+    assert f(None, None, None, 0, 64, 64, 64, None, 8, 8, 1, 512, BF16, BF16, 1e-6, None) == OK
+
+
+def test_qkv_norm_proj_validation(lib):
+    f = lib.qkv_norm_proj
+    # (x, Wf, y, M, K, nq, nk, nv, wq, wk, wv, wdt, eps, n_seg, stream)
+    assert f(P, P, P, 8, 64, 64, 32, 32, P, P, None, BF16, 1e-6, 1, None) == NULL     # wv with nv > 0
+    assert f(P, P, P, 8, 60, 64, 32, 32, P, P, P, BF16, 1e-6, 1, None) == SHAPE       # K % 8
+    assert f(P, P, P, 8, 64, 64, 32, 30, P, P, P, BF16, 1e-6, 1, None) == SHAPE       # N % 8
+    assert f(P, P, P, 8, 64, 64, 32, 32, P, P, P, BF16, 1e-6, 3, None) == SHAPE       # n_seg
+    assert f(P, P, P, 8, 64, 64, 32, 32, P, P, P, BF16, float("nan"), 1, None) == EPS
+    assert f(P + 8, P, P, 8, 64, 64, 32, 32, P, P, P, BF16, 1e-6, 1, None) == ALIGN

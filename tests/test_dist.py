@@ -89,3 +89,34 @@ def test_shard_rows_rejects_bad_requests():
 
 def test_max_without_process_group_is_identity():
     assert qdist.max_over_ranks(3.5) == 3.5
+
+
+def _gather_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from rmsnorm_qknorm_b200.tp import gather_partials
+        local = torch.arange(5, dtype=torch.float32) + 100 * rank  # this rank's per-row partials
+        g = gather_partials(local)
+        out[rank] = g.tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_scalar_partials_all_gather_rank_order():
+    # tensor-parallel QK-Norm exchanges only [rows] fp32 per rank; the gathered
+    # [world, rows] array is in rank order on every rank (the fixed combine order)
+    world, port = 2, _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_gather_worker, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    expect = [[float(i) for i in range(5)], [100.0 + i for i in range(5)]]
+    assert res[0] == expect and res[1] == expect
+
+
+def test_gather_without_process_group_is_local():
+    from rmsnorm_qknorm_b200.tp import gather_partials
+    g = gather_partials(torch.ones(3))
+    assert tuple(g.shape) == (1, 3)

@@ -279,3 +279,24 @@ def test_round_bf16_ties_and_double_rounding():
 
 def test_oracle_threads_positive():
     assert oracle.threads() >= 1
+
+
+# --------------------------------------------------------------- RMSNorm elimination
+
+
+@pytest.mark.parametrize("eps_post", [0.0, 1e-6])
+def test_rmsnorm_elimination_identity(eps_post):
+    # FlashNorm (abstract): RMSNorm -> linear -> RMSNorm lets the first RMSNorm go.
+    # With the first norm's eps = 0, RMSNorm(RMSNorm(x; w) W; v) = RMSNorm((x diag(w)) W; v)
+    # because the first norm only scales each row of the product by 1/rms(x) > 0.
+    x, w, W, v = rand(6, 40), rand(40), rand(40, 24), rand(24)
+    full = oracle.rmsnorm(oracle.norm_then_project(x, w, W, 0.0), v, eps_post)
+    eliminated = oracle.rmsnorm(x @ oracle.fold_weights(w, W), v, eps_post)  # numpy matmul: a library step
+    tol = 1e-12 if eps_post == 0.0 else 1e-6
+    np.testing.assert_allclose(eliminated, full, rtol=tol, atol=1e-12)
+
+
+def test_rmsnorm_elimination_needs_the_second_norm():
+    # without the second norm the row scale 1/rms(x) survives: catches an identity applied too widely
+    x, w, W = rand(4, 16) * 5, rand(16), rand(16, 8)
+    assert not np.allclose(oracle.norm_then_project(x, w, W, 0.0), x @ oracle.fold_weights(w, W))

@@ -50,14 +50,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  After
-// kWaitTimeoutNs it stores 1 into *err and returns false.
-__device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, int *err) {
+// timeout_ns it stores 1 into *err and returns false.
+__device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, int *err,
+                                              uint64_t timeout_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer();
     while (true) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer() - t0 > kWaitTimeoutNs) {
+        if (global_timer() - t0 > timeout_ns) {
             atomicExch(err, 1);
             return false;
         }

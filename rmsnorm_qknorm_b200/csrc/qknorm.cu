@@ -256,6 +256,8 @@ struct Args {
     int stages;       // W * stages per warp
     int stage_bytes;  // multiple of 16
     int w_bytes;      // fp32 weights of both jobs
+    uint64_t wait_ns;  // limit of every mbarrier wait
+    int fault_warp;   // testing only: this block*W+warp skips its first tile's copies (-1: none)
 };
 
 // Shared memory: [ring][fp32 weights][full bars][W x 8 x 32 floats scratch]
@@ -538,7 +540,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
         for (int j = 0; j < spw; ++j) {
             const int64_t tile = first + j * step;
             if (tile >= a.total_tiles) break;
-            issue_tile(a, tile, nt0, smem + (size_t)(warp * spw + j) * SB, &full[warp * spw + j]);
+            // (testing only) an injected fault: the copies are never issued, so
+            // this stage's wait cannot complete and must give up on its own
+            if (!(j == 0 && a.fault_warp == (int)blockIdx.x * W + warp))
+                issue_tile(a, tile, nt0, smem + (size_t)(warp * spw + j) * SB, &full[warp * spw + j]);
             ++issued;
         }
     }
@@ -586,7 +591,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
         const int slot = (int)(k % spw);
         const int stage = warp * spw + slot;
         const uint32_t par = (uint32_t)(k / spw) & 1u;
-        if (!mbar_wait(smem_u32(&full[stage]), par, &g_norm_error)) break;
+        if (!mbar_wait(smem_u32(&full[stage]), par, &g_norm_error, a.wait_ns)) break;
         const int which = tile >= nt0 ? 1 : 0;
         const Job J = pick(a, which);
         const int64_t row0 = (tile - (which ? nt0 : 0)) * J.rows_per_tile;
@@ -611,7 +616,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
     // drain: copies this warp issued but did not consume (only after a failed
     // wait) must land before the block exits
     for (; k < issued; ++k)
-        mbar_wait(smem_u32(&full[warp * spw + (int)(k % spw)]), (uint32_t)(k / spw) & 1u, &g_norm_error);
+        mbar_wait(smem_u32(&full[warp * spw + (int)(k % spw)]), (uint32_t)(k / spw) & 1u, &g_norm_error, a.wait_ns);
 }
 
 }  // namespace staged
@@ -717,6 +722,10 @@ bool staged_geometry(int64_t max_row_bytes, int64_t w_bytes, int *warps, int *sp
     return false;
 }
 
+// One-shot fault injection for testing the bounded waits (this host thread's
+// next staged-kernel launch); see qkn_testing_arm_wait_fault.
+thread_local uint64_t t_fault_wait_ns = 0;
+
 template <typename TA, typename TW, bool STATS>
 qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps, float *partial,
                          int warps, int spw, int stage_bytes, cudaStream_t s) {
@@ -731,6 +740,13 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     a.stages = warps * spw;
     a.stage_bytes = stage_bytes;
     a.w_bytes = 0;
+    a.wait_ns = kWaitTimeoutNs;
+    a.fault_warp = -1;
+    if (t_fault_wait_ns != 0) {
+        a.wait_ns = t_fault_wait_ns;
+        a.fault_warp = 0;
+        t_fault_wait_ns = 0;
+    }
     for (int i = 0; i < njobs; ++i) {
         const Tensor2 &t = ts[i];
         staged::Job &J = a.job[i];
@@ -1055,4 +1071,11 @@ extern "C" QKN_API qkn_status rmsnorm_apply_partials(const void *x, const void *
                                                   part_stride, d_full, eps, s);
     return launch_apply<float, float>(x, w, y, rows, d, ld, ld_out, partial, n_part, part_row_stride, part_stride,
                                       d_full, eps, s);
+}
+
+extern "C" QKN_API qkn_status qkn_testing_arm_wait_fault(uint64_t wait_ns) {
+    if (wait_ns == 0 || wait_ns > qkn::kWaitTimeoutNs)
+        return qkn::fail(QKN_ERR_SHAPE, "qkn_testing_arm_wait_fault: wait_ns must be in (0, 2e9]");
+    qkn::t_fault_wait_ns = wait_ns;
+    return QKN_OK;
 }

@@ -161,3 +161,9 @@ def test_qkv_norm_proj_validation(lib):
     assert f(P, P, P, 8, 64, 64, 32, 32, P, P, P, BF16, 1e-6, 3, None) == SHAPE       # n_seg
     assert f(P, P, P, 8, 64, 64, 32, 32, P, P, P, BF16, float("nan"), 1, None) == EPS
     assert f(P + 8, P, P, 8, 64, 64, 32, 32, P, P, P, BF16, 1e-6, 1, None) == ALIGN
+
+
+def test_fault_hook_validation(lib):
+    lib.qkn_testing_arm_wait_fault.argtypes = [ctypes.c_uint64]
+    assert lib.qkn_testing_arm_wait_fault(0) == SHAPE
+    assert lib.qkn_testing_arm_wait_fault(3_000_000_000) == SHAPE

@@ -409,6 +409,254 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
 
 }  // namespace gemm
 
+// ============================================ tcgen05 GEMM, CTA pair (ii)
+//
+// The same projection on a cluster of two CTAs (two SMs of a TPC) that
+// compute one 256 x 256 tile together with tcgen05.mma.cta_group::2: each CTA
+// keeps its own 128 rows of x and its own 128 rows of W' for a k-block in
+// shared memory (32 KiB per stage instead of 48), the even CTA issues the
+// M = 256 MMAs that read both CTAs' tiles, and each CTA's tensor memory holds
+// the fp32 accumulator of its own 128 rows.  Per SM that is a third less
+// shared-memory traffic per FLOP, and six stages fit.  Both CTAs' TMA loads
+// complete their bytes on the even CTA's stage barrier; the even CTA's
+// commits arrive (multicast) on the stage and accumulator barriers of both
+// CTAs; the epilogue warps of both CTAs release the even CTA's accumulator
+// barrier.  The x tiles of the pair are also the rows the CTAs scale, so the
+// epilogue is the same as the single-CTA kernel's, with a 1/rms supplied.
+namespace gemm2 {
+
+constexpr int BM = 128;                                  // rows per CTA (256 per pair)
+constexpr int BN = 256;                                  // columns per pair tile
+constexpr int BN_CTA = 128;                              // W' rows loaded by each CTA
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;                     // 16 KiB
+constexpr int B_BYTES = BN_CTA * BK * 2;                 // 16 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 32 KiB per CTA
+constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;        // bytes landing on the even CTA's barrier
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int THREADS = 192;                             // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int GROUP_M = 8;                               // pair row blocks (of 256) per raster group
+
+static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 D, M = 256, N = 256.
+constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                ((uint32_t)(256 >> 4) << 24);
+
+struct Args {
+    const float *inv_rms;  // [M] 1/rms of every row (nullptr with unit_scale)
+    __nv_bfloat16 *y;      // [M][N]
+    int M, N, K;
+    int pm_blocks, n_blocks, k_blocks, num_tiles;  // pm: 256-row blocks of the pair
+    int unit_scale;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, const Args &g, int &pm, int &n) {
+    const int group_tiles = GROUP_M * g.n_blocks;
+    const int group = tile / group_tiles;
+    const int first = group * GROUP_M;
+    const int rows_in_group = min(g.pm_blocks - first, GROUP_M);
+    const int in_group = tile - group * group_tiles;
+    pm = first + in_group % rows_in_group;
+    n = in_group / rows_in_group;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 2-D tensor copy into this CTA's shared memory whose bytes complete on the
+// barrier at `bar_cluster` (the even CTA's), for a CTA-pair MMA.  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kInstrDesc), "r"(accumulate));
+}
+
+// Arrives, once these MMAs have completed, on the barrier at this offset in
+// both CTAs of the pair.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+    const uint16_t mask = 0x3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(bar), "h"(mask) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                           const Args g) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + STAGES;
+    uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);   // even CTA: its producer's arrive + both CTAs' bytes
+            mbar_init(smem_u32(&empty[s]), 1);  // the even CTA's multicast commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&acc_full[a]), 1);   // the even CTA's multicast commit
+            mbar_init(smem_u32(&acc_empty[a]), 8);  // even CTA: 4 epilogue warps of each CTA
+        }
+        mbar_init_fence();
+    }
+    if (warp == 1) {  // whole warp, in both CTAs: the pair's tensor memory
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    gemm::tc_fence_before();
+    cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
+    gemm::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < g.num_tiles; tile += num_pairs) {
+            int pm, n;
+            tile_coords(tile, g, pm, n);
+            for (int kb = 0; kb < g.k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &g_device_error)) { ok = false; break; }
+                if (lane == 0) {
+                    const uint32_t fb_local = smem_u32(&full[stage]);
+                    const uint32_t fb = map_to_rank(fb_local, 0);
+                    if (leader) mbar_arrive_expect_tx(fb_local, PAIR_STAGE_BYTES);
+                    uint8_t *sa = smem + stage * STAGE_BYTES;
+                    tma_load_2d_pair(smem_u32(sa), &tmap_x, kb * BK, pm * 2 * BM + (int)rank * BM, fb);
+                    tma_load_2d_pair(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, n * BN + (int)rank * BN_CTA, fb);
+                }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer (even CTA)
+        if (leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < g.num_tiles; tile += num_pairs, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, &g_device_error)) break;
+                gemm::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
+                    gemm::tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+                        const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                        for (int k = 0; k < BK / gemm::UMMA_K; ++k)
+                            umma_pair(d_tmem, gemm::sw128_kmajor_desc(a0 + k * 32),
+                                      gemm::sw128_kmajor_desc(b0 + k * 32), (kb | k) != 0 ? 1u : 0u);
+                        umma_commit_pair(smem_u32(&empty[stage]));  // frees the stage in both CTAs
+                    }
+                    __syncwarp();
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                if (lane == 0) umma_commit_pair(smem_u32(&acc_full[acc]));  // both CTAs' accumulators ready
+                __syncwarp();
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2..5, both CTAs)
+        const int quarter = warp & 3;
+        int it = 0;
+        for (int tile = pair; tile < g.num_tiles; tile += num_pairs, ++it) {
+            int pm, n;
+            tile_coords(tile, g, pm, n);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase, &g_device_error)) break;
+            gemm::tc_fence_after();
+            const int row = pm * 2 * BM + (int)rank * BM + quarter * 32 + lane;
+            const bool row_ok = row < g.M;
+            const float r = g.unit_scale ? 1.f : (row_ok ? __ldg(g.inv_rms + row) : 0.f);
+            __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                gemm::tmem_ld_32cols(tbase + c * 32, v);
+                const int col0 = n * BN + c * 32;
+                if (row_ok) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int col = col0 + j * 8;
+                        if (col < g.N) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * r, __uint_as_float(v[8 * j + 1]) * r);
+                            o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * r, __uint_as_float(v[8 * j + 3]) * r);
+                            o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * r, __uint_as_float(v[8 * j + 5]) * r);
+                            o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * r, __uint_as_float(v[8 * j + 7]) * r);
+                            *reinterpret_cast<uint4 *>(yrow + col) = o;
+                        }
+                    }
+                }
+            }
+            gemm::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&acc_empty[acc]), 0));
+        }
+    }
+
+    gemm::tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the even CTA's MMAs (which read this CTA's tiles) are done in both CTAs
+    if (warp == 1) {
+        gemm::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace gemm2
+
 // ----------------------------------------------------------- host helpers
 
 namespace {
@@ -453,10 +701,49 @@ qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float
     return check_launch("inv_rms_kernel launch");
 }
 
-// inv == nullptr: the kernel computes every row's 1/rms itself (eps) and,
-// when inv_out is given, stores it there.
+#ifndef QKN_GEMM_PAIR
+#define QKN_GEMM_PAIR 1
+#endif
+
+// The CTA-pair projection: inv (1/rms per row) given, or unit_scale.
+qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N,
+                            int64_t K, bool unit_scale, cudaStream_t s) {
+    CUtensorMap tx, tw;
+    if (qkn_status st = make_tmap(&tx, x, M, K, gemm2::BM)) return st;
+    if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm2::BN_CTA)) return st;
+    gemm2::Args g;
+    g.inv_rms = inv;
+    g.y = static_cast<__nv_bfloat16 *>(y);
+    g.M = (int)M;
+    g.N = (int)N;
+    g.K = (int)K;
+    g.pm_blocks = (int)((M + 2 * gemm2::BM - 1) / (2 * gemm2::BM));
+    g.n_blocks = (int)((N + gemm2::BN - 1) / gemm2::BN);
+    g.k_blocks = (int)((K + gemm2::BK - 1) / gemm2::BK);
+    g.num_tiles = g.pm_blocks * g.n_blocks;
+    g.unit_scale = unit_scale ? 1 : 0;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm2::flashnorm_gemm_pair_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(flashnorm_gemm_pair_kernel)");
+        attr_set[dev] = true;
+    }
+    const int pairs = sm_count() / 2;
+    const int grid = 2 * (g.num_tiles < pairs ? g.num_tiles : pairs);
+    gemm2::flashnorm_gemm_pair_kernel<<<grid, gemm2::THREADS, gemm2::SMEM_BYTES, s>>>(tx, tw, g);
+    return check_launch("flashnorm_gemm_pair_kernel launch");
+}
+
+// inv == nullptr (and not unit_scale): the single-CTA kernel computes every
+// row's 1/rms itself (eps) and, when inv_out is given, stores it there.
+// Otherwise the CTA-pair kernel runs with the given 1/rms (or none).
 qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
                        float eps, float *inv_out, cudaStream_t s, bool unit_scale = false) {
+    if (QKN_GEMM_PAIR && (inv != nullptr || unit_scale))
+        return launch_gemm_pair(x, Wf, y, inv, M, N, K, unit_scale, s);
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;

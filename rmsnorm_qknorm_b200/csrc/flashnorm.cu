@@ -436,9 +436,10 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 32 KiB per CTA
 constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;        // bytes landing on the even CTA's barrier
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int THREADS = 192;                             // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-7 row statistics
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int INV_BYTES = 2 * BM * 4;                     // 1/rms of this CTA's rows, both accumulators
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + INV_BYTES + 1024;
 constexpr int GROUP_M = 8;                               // pair row blocks (of 256) per raster group
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
@@ -449,11 +450,14 @@ constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
                                 ((uint32_t)(256 >> 4) << 24);
 
 struct Args {
-    const float *inv_rms;  // [M] 1/rms of every row (nullptr with unit_scale)
+    const float *inv_rms;  // [M] given 1/rms (compute_inv == 0 and unit_scale == 0)
+    float *inv_out;        // [M] optional: receives the 1/rms computed in-kernel
     __nv_bfloat16 *y;      // [M][N]
     int M, N, K;
     int pm_blocks, n_blocks, k_blocks, num_tiles;  // pm: 256-row blocks of the pair
     int unit_scale;
+    int compute_inv;       // 1: each CTA computes its rows' 1/rms from its x tiles
+    float eps;
 };
 
 __device__ __forceinline__ void tile_coords(int tile, const Args &g, int &pm, int &n) {
@@ -481,6 +485,29 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
 
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// try_wait with cluster-scope acquire: for phases completed by the peer CTA.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int *err) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (global_timer() - t0 > kWaitTimeoutNs) {
+            atomicExch(err, 1);
+            return false;
+        }
+    }
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
@@ -520,7 +547,11 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+    uint64_t *stats_ready = bars + 2 * STAGES + 4;       // odd CTA: its x tile of a stage has landed
+    uint64_t *stats_full = bars + 3 * STAGES + 4;        // this CTA's 1/rms of an accumulator published
+    uint64_t *inv_free = bars + 3 * STAGES + 6;          // this CTA's epilogue is done with an inv buffer
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 8);
+    float *inv_buf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);  // [2][BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -530,11 +561,15 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 1);   // even CTA: its producer's arrive + both CTAs' bytes
-            mbar_init(smem_u32(&empty[s]), 1);  // the even CTA's multicast commit
+            // the even CTA's multicast commit, plus this CTA's statistics warps when they read x
+            mbar_init(smem_u32(&empty[s]), g.compute_inv ? 3 : 1);
+            mbar_init(smem_u32(&stats_ready[s]), 1);  // odd CTA: relayed by the even CTA's MMA warp
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&acc_full[a]), 1);   // the even CTA's multicast commit
             mbar_init(smem_u32(&acc_empty[a]), 8);  // even CTA: 4 epilogue warps of each CTA
+            mbar_init(smem_u32(&stats_full[a]), 2); // this CTA's two statistics warps
+            mbar_init(smem_u32(&inv_free[a]), 4);   // this CTA's four epilogue warps
         }
         mbar_init_fence();
     }
@@ -587,6 +622,8 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
                     if (!mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
                     gemm::tc_fence_after();
                     if (lane == 0) {
+                        // both CTAs' tiles of this stage have landed: tell the odd CTA's statistics warps
+                        if (g.compute_inv) mbar_arrive_cluster(map_to_rank(smem_u32(&stats_ready[stage]), 1));
                         const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
                         const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
@@ -603,7 +640,7 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
                 __syncwarp();
             }
         }
-    } else {
+    } else if (warp < 6) {
         // ---------------------------------------------------------------- epilogue (warps 2..5, both CTAs)
         const int quarter = warp & 3;
         int it = 0;
@@ -616,7 +653,15 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
             gemm::tc_fence_after();
             const int row = pm * 2 * BM + (int)rank * BM + quarter * 32 + lane;
             const bool row_ok = row < g.M;
-            const float r = g.unit_scale ? 1.f : (row_ok ? __ldg(g.inv_rms + row) : 0.f);
+            float r;
+            if (g.unit_scale) {
+                r = 1.f;
+            } else if (g.compute_inv) {
+                if (!mbar_wait(smem_u32(&stats_full[acc]), acc_phase, &g_device_error)) break;
+                r = inv_buf[acc * BM + quarter * 32 + lane];
+            } else {
+                r = row_ok ? __ldg(g.inv_rms + row) : 0.f;
+            }
             __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll 1
@@ -641,7 +686,70 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
             }
             gemm::tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&acc_empty[acc]), 0));
+            if (lane == 0) {
+                if (g.compute_inv) mbar_arrive(smem_u32(&inv_free[acc]));
+                mbar_arrive_cluster(map_to_rank(smem_u32(&acc_empty[acc]), 0));
+            }
+        }
+    } else if (g.compute_inv) {
+        // ---------------------------------------------------------------- row statistics (warps 6, 7)
+        // Each CTA sums the squares of its own 128 x rows over K from the x
+        // tiles streaming through its shared memory (the 128-byte swizzle
+        // only permutes the 16-byte chunks inside a row).  Lane l of warp sw
+        // owns rows sw*64 + l and sw*64 + l + 32.  The even CTA waits on its
+        // stage barrier; the odd CTA on the relay its MMA warp sends.
+        const int sw = warp - 6;
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < g.num_tiles; tile += num_pairs, ++it) {
+            int pm, n;
+            tile_coords(tile, g, pm, n);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            float2 ssq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            for (int kb = 0; kb < g.k_blocks; ++kb) {
+                const bool landed = leader ? mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)
+                                           : mbar_wait_cluster(smem_u32(&stats_ready[stage]), phase, &g_device_error);
+                if (!landed) { ok = false; break; }
+                const uint8_t *a_tile = smem + stage * STAGE_BYTES;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int rr = sw * 64 + lane + 32 * i;
+                    const uint8_t *arow = a_tile + rr * (BK * 2);
+                    uint4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4 *>(arow + ((j ^ (rr & 7)) * 16));
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float2 p0 = make_float2(bf16lo(v[j].x), bf16hi(v[j].x));
+                        const float2 p1 = make_float2(bf16lo(v[j].y), bf16hi(v[j].y));
+                        const float2 p2 = make_float2(bf16lo(v[j].z), bf16hi(v[j].z));
+                        const float2 p3 = make_float2(bf16lo(v[j].w), bf16hi(v[j].w));
+                        ssq[i] = __ffma2_rn(p0, p0, ssq[i]);
+                        ssq[i] = __ffma2_rn(p1, p1, ssq[i]);
+                        ssq[i] = __ffma2_rn(p2, p2, ssq[i]);
+                        ssq[i] = __ffma2_rn(p3, p3, ssq[i]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[stage]));
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            // the inv buffer of this accumulator is free once this CTA's epilogue finished tile it - 2
+            if (!mbar_wait(smem_u32(&inv_free[acc]), acc_phase ^ 1u, &g_device_error)) break;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int rr = sw * 64 + lane + 32 * i;
+                const float inv = rsqrtf((ssq[i].x + ssq[i].y) / (float)g.K + g.eps);
+                inv_buf[acc * BM + rr] = inv;
+                const int row = pm * 2 * BM + (int)rank * BM + rr;
+                if (g.inv_out != nullptr && n == 0 && row < g.M) g.inv_out[row] = inv;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&stats_full[acc]));
         }
     }
 
@@ -701,13 +809,15 @@ qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float
     return check_launch("inv_rms_kernel launch");
 }
 
+// The CTA-pair kernel measured slower than the single-CTA kernel in same-box
+// A/B runs, so it is not the default; QKN_GEMM_PAIR=1 selects it.
 #ifndef QKN_GEMM_PAIR
-#define QKN_GEMM_PAIR 1
+#define QKN_GEMM_PAIR 0
 #endif
 
 // The CTA-pair projection: inv (1/rms per row) given, or unit_scale.
 qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N,
-                            int64_t K, bool unit_scale, cudaStream_t s) {
+                            int64_t K, bool unit_scale, float eps, float *inv_out, cudaStream_t s) {
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm2::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm2::BN_CTA)) return st;
@@ -722,6 +832,9 @@ qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float 
     g.k_blocks = (int)((K + gemm2::BK - 1) / gemm2::BK);
     g.num_tiles = g.pm_blocks * g.n_blocks;
     g.unit_scale = unit_scale ? 1 : 0;
+    g.compute_inv = (inv == nullptr && !unit_scale) ? 1 : 0;
+    g.inv_out = g.compute_inv ? inv_out : nullptr;
+    g.eps = eps;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -731,7 +844,30 @@ qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float 
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(flashnorm_gemm_pair_kernel)");
         attr_set[dev] = true;
     }
-    const int pairs = sm_count() / 2;
+    // a persistent grid must fit at once: as many pairs as the device can
+    // keep resident together (two-SM clusters need both SMs of a pair free)
+    static int max_clusters[64] = {0};
+    if (dev >= 0 && dev < 64 && max_clusters[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+        cfg.blockDim = dim3(gemm2::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gemm2::SMEM_BYTES;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm2::flashnorm_gemm_pair_kernel, &cfg);
+        if (e != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = sm_count() / 2;
+        }
+        max_clusters[dev] = n;
+    }
+    const int pairs = (dev >= 0 && dev < 64) ? max_clusters[dev] : sm_count() / 2;
     const int grid = 2 * (g.num_tiles < pairs ? g.num_tiles : pairs);
     gemm2::flashnorm_gemm_pair_kernel<<<grid, gemm2::THREADS, gemm2::SMEM_BYTES, s>>>(tx, tw, g);
     return check_launch("flashnorm_gemm_pair_kernel launch");
@@ -739,11 +875,14 @@ qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float 
 
 // inv == nullptr (and not unit_scale): the single-CTA kernel computes every
 // row's 1/rms itself (eps) and, when inv_out is given, stores it there.
-// Otherwise the CTA-pair kernel runs with the given 1/rms (or none).
+// The CTA-pair kernel serves every form; the single-CTA kernel is the
+// fallback when a two-CTA cluster cannot be launched on the device.
 qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
                        float eps, float *inv_out, cudaStream_t s, bool unit_scale = false) {
-    if (QKN_GEMM_PAIR && (inv != nullptr || unit_scale))
-        return launch_gemm_pair(x, Wf, y, inv, M, N, K, unit_scale, s);
+    if (QKN_GEMM_PAIR && sm_count() >= 2) {
+        const qkn_status st = launch_gemm_pair(x, Wf, y, inv, M, N, K, unit_scale, eps, inv_out, s);
+        if (st != QKN_ERR_CUDA) return st;  // a launch the device refused falls through
+    }
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;

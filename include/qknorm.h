@@ -24,6 +24,7 @@
 #ifndef QKNORM_H
 #define QKNORM_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -95,6 +96,29 @@ QKN_API qkn_status qknorm_fused(const void *q, const void *k,
                                 int64_t ldq_out, int64_t ldk_out,
                                 qkn_dtype act, qkn_dtype wdt,
                                 float eps, int n_seg, void *stream);
+
+/*
+ * qknorm_fused_host -- qknorm_fused on rows held in HOST memory.
+ *
+ * Same computation as qknorm_fused (SwiftQK, abstract), for q [T][dq] and
+ * k [T][dk] in host memory (contiguous rows; pinned memory lets the copies
+ * run at full link speed).  The rows stream through `workspace` (device, at
+ * least 3 x (dq + dk) x element size bytes, 256-byte aligned) in chunks on
+ * three internal streams that take chunks in turn, so the upload of one
+ * chunk, the kernel of another and the download of a third overlap.  Results
+ * land in q_out / k_out (host, may equal q / k).  wq, wk are DEVICE pointers.
+ * The work is ordered after what is already on `stream`, and `stream` waits
+ * for it: the call returns before the copies finish, so the host buffers must
+ * stay valid (and unread) until `stream` has been synchronised.  dk == 0
+ * normalises q only.  The internal streams are created on the first call per
+ * device and kept until exit.
+ */
+QKN_API qkn_status qknorm_fused_host(const void *q, const void *k,
+                                     const void *wq, const void *wk,
+                                     void *q_out, void *k_out,
+                                     int64_t T, int64_t dq, int64_t dk,
+                                     qkn_dtype act, qkn_dtype wdt, float eps, int n_seg,
+                                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * rmsnorm_partial_stats -- the per-shard scalar statistics on their own.

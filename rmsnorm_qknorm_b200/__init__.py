@@ -88,8 +88,10 @@ def load_library() -> ctypes.CDLL:
         lib.rmsnorm_apply_partials.argtypes = [p, p, p, i64, i64, i64, i64, p, i32, i64, i64, i64,
                                                i32, i32, f32, p]
         lib.qkv_norm_proj.argtypes = [p, p, p, i64, i64, i64, i64, i64, p, p, p, i32, f32, i32, p]
+        lib.qknorm_fused_host.argtypes = [p, p, p, p, p, p, i64, i64, i64, i32, i32, f32, i32,
+                                          p, ctypes.c_size_t, p]
         lib.qkn_check_device.argtypes = [p]
-        for f in ("qknorm_fused", "rmsnorm_partial_stats", "flashnorm_fold_weights",
+        for f in ("qknorm_fused", "qknorm_fused_host", "rmsnorm_partial_stats", "flashnorm_fold_weights",
                   "flashnorm_proj", "rmsnorm_apply_partials", "qkv_norm_proj", "qkn_check_device"):
             getattr(lib, f).restype = ctypes.c_int
         lib.qkn_last_error.restype = ctypes.c_char_p
@@ -190,6 +192,67 @@ def qknorm_fused(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
                           act, wdt, float(eps), int(n_seg), _stream(stream))
     _check("qknorm_fused", st)
     return q_out_t, k_out_t
+
+
+HOST_WORKSPACE_BYTES = 3 * 32 * 1024 * 1024
+
+
+def qknorm_fused_host(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
+                      wk: torch.Tensor | None, eps: float = 1e-6, n_seg: int = 1, *,
+                      q_out: torch.Tensor | None = None, k_out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, stream=None):
+    """QK-Norm of q [T, dq] and k [T, dk] held in HOST memory; results in host tensors.
+
+    The rows stream through a device ``workspace`` (uint8 CUDA tensor,
+    ``HOST_WORKSPACE_BYTES`` allocated when not given) in chunks whose upload,
+    kernel and download overlap.  wq / wk live on the device.  Pinned host
+    tensors let the copies run at link speed.  The call is asynchronous on
+    ``stream``: synchronise it before reading the outputs.  Returns
+    ``(q_out, k_out)``; ``q_out=q`` works in place.
+    """
+    def host_rows(t, name):
+        if not isinstance(t, torch.Tensor) or t.is_cuda:
+            raise ValueError(f"{name} must be a host (CPU) tensor")
+        if t.dim() != 2 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 2-D tensor")
+        return t.shape
+    T, dq = host_rows(q, "q")
+    act = _dtype_code(q.dtype)
+    _vec(wq, "wq", dq)
+    wdt = _dtype_code(wq.dtype)
+    if k is not None:
+        Tk, dk = host_rows(k, "k")
+        if Tk != T or k.dtype != q.dtype:
+            raise ValueError("k must have q's row count and dtype")
+        if wk is None:
+            raise ValueError("wk is required with k")
+        _vec(wk, "wk", dk)
+        if wk.dtype != wq.dtype:
+            raise ValueError("wk must have wq's dtype")
+    else:
+        dk = 0
+    pin = q.is_pinned()
+    if q_out is None:
+        q_out = torch.empty((T, dq), dtype=q.dtype, pin_memory=pin)
+    if host_rows(q_out, "q_out") != (T, dq) or q_out.dtype != q.dtype:
+        raise ValueError("q_out must match q")
+    if k is not None:
+        if k_out is None:
+            k_out = torch.empty((T, dk), dtype=k.dtype, pin_memory=pin)
+        if host_rows(k_out, "k_out") != (T, dk) or k_out.dtype != k.dtype:
+            raise ValueError("k_out must match k")
+    if workspace is None:
+        workspace = torch.empty(HOST_WORKSPACE_BYTES, dtype=torch.uint8, device=wq.device)
+    _cuda(workspace, "workspace")
+    lib = load_library()
+    st = lib.qknorm_fused_host(q.data_ptr(), k.data_ptr() if k is not None else None,
+                               wq.data_ptr(), wk.data_ptr() if k is not None else None,
+                               q_out.data_ptr(), k_out.data_ptr() if k is not None else None,
+                               T, dq, dk, act, wdt, float(eps), int(n_seg),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               _stream(stream))
+    _check("qknorm_fused_host", st)
+    return q_out, (k_out if k is not None else None)
 
 
 def rmsnorm_partial_stats(x: torch.Tensor, n_seg: int, *, out: torch.Tensor | None = None,

@@ -167,3 +167,24 @@ def test_fault_hook_validation(lib):
     lib.qkn_testing_arm_wait_fault.argtypes = [ctypes.c_uint64]
     assert lib.qkn_testing_arm_wait_fault(0) == SHAPE
     assert lib.qkn_testing_arm_wait_fault(3_000_000_000) == SHAPE
+
+
+def test_host_entry_validation(lib):
+    # qknorm_fused_host(q, k, wq, wk, q_out, k_out, T, dq, dk, act, wdt, eps, n_seg, ws, ws_bytes, stream)
+    f = lib.qknorm_fused_host
+    big = 1 << 20
+
+    def h(q=P, k=P, wq=P, wk=P, qo=P, ko=P, T=4, dq=64, dk=64, act=BF16, wdt=BF16, eps=1e-6, n_seg=1,
+          ws=P, nbytes=big):
+        return f(q, k, wq, wk, qo, ko, T, dq, dk, act, wdt, eps, n_seg, ws, nbytes, None)
+
+    assert h(ws=None) == NULL
+    assert h(k=None) == NULL
+    assert h(T=-1) == SHAPE
+    assert h(dq=60, n_seg=8) == SHAPE
+    assert h(act=5) == DTYPE
+    assert h(eps=float("nan")) == EPS
+    assert h(nbytes=3 * 255) == SHAPE          # not even one row per stream buffer
+    assert "workspace" in lib.qkn_last_error().decode()
+    assert h(ws=P + 16) == ALIGN               # workspace must be 256-byte aligned
+    assert h(T=0, q=None, k=None, qo=None, ko=None, ws=None) == OK

@@ -498,7 +498,8 @@ def run_flashnorm(args, rank, world, local, pg):
     value = world * wl.M / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
     tflops = wl.flops() / (avg_gemm * 1e-3) / 1e12
-    src = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
+    src = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
+           "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
            "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
 
     e2e = None

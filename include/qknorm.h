@@ -214,6 +214,49 @@ QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded, void *y,
                                   void *stream);
 
 /*
+ * qkv_proj_qknorm -- RMSNorm, QKV projection and QK-Norm in one GEMM: the
+ * normalised q and k are formed in the projection's epilogue and never
+ * travel through HBM unnormalised.
+ *
+ * Defined by: FlashNorm, abstract (fold the input norm's weights into W',
+ * apply the scalar 1/rms to the matmul output) and SwiftQK, abstract (the
+ * QK-Norm factor depends on a token's full query / key vector; the pieces of
+ * that vector held in different places contribute scalar partial sums of
+ * squares, combined in a fixed order):
+ *   u[m][n]              = r[m] * sum_k x[m][k] W'[n][k]      fp32 accumulate
+ *   y[m][0:nq)           = RMSNorm(u[m][0:nq);  wq, eps_qk)
+ *   y[m][nq:nq+nk)       = RMSNorm(u[m][nq:nq+nk); wk, eps_qk)
+ *   y[m][nq+nk:nq+nk+nv) = u[m][nq+nk:nq+nk+nv)
+ * with RMSNorm(v; w, e)_i = (v_i * 1/sqrt(mean(v^2) + e)) * w_i in fp32 and
+ * one RNE rounding to bf16.  A row's q (k) statistic is the sum, in tile
+ * order, of its per-256-column-tile partial sums, exchanged between the
+ * CTAs of one kernel.
+ *
+ * r[m]: inv_rms given -> used as given; inv_rms NULL and inv_rms_out given
+ * -> a statistics pass writes 1/sqrt(mean(x[m]^2) + eps) there first; both
+ * NULL -> r = 1 (x used as it is, e.g. already normalised).
+ *
+ * x [M][K] bf16; W_folded [nq+nk+nv][K] bf16 (K contiguous, from
+ * flashnorm_fold_weights with out_k_major = 1); y [M][nq+nk+nv] bf16; wq
+ * [nq], wk [nk] of dtype wdt.  K, nq, nk, nv multiples of 8 (nv may be 0);
+ * x, W_folded, y, wq, wk, workspace 16-byte aligned.  workspace: device
+ * scratch of at least qkv_proj_qknorm_workspace_bytes(M, nq, nk, nv) bytes,
+ * or NULL to allocate it stream-ordered inside the call.  The kernel is
+ * launched cooperatively (all its CTAs resident at once); QKN_ERR_UNSUPPORTED
+ * when nq or nk spans more 256-column tiles than the device has SMs.  A
+ * device-side wait that gives up is reported by qkn_check_device.
+ */
+QKN_API qkn_status qkv_proj_qknorm(const void *x, const void *W_folded, void *y,
+                                   int64_t M, int64_t K, int64_t nq, int64_t nk, int64_t nv,
+                                   const void *wq, const void *wk, qkn_dtype wdt,
+                                   float eps, float eps_qk,
+                                   const float *inv_rms, float *inv_rms_out,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace qkv_proj_qknorm needs (0 for invalid sizes). */
+QKN_API size_t qkv_proj_qknorm_workspace_bytes(int64_t M, int64_t nq, int64_t nk, int64_t nv);
+
+/*
  * qkv_norm_proj -- QKV projection with QKV-normalisation, pre-attention
  * RMSNorm eliminated.
  *

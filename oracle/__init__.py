@@ -154,6 +154,23 @@ def flashnorm_deferred(x, Wf, eps: float) -> np.ndarray:
     return out
 
 
+def qkv_proj_qknorm(x, w_in, W, wq, wk, nq: int, nk: int, eps: float, eps_qk: float,
+                    input_norm: bool = True) -> np.ndarray:
+    """Pre-attention path: u = RMSNorm(x; w_in, eps) @ W (or x @ W without the
+    input norm), then QK-Norm of the first nq columns (weights wq) and of the
+    next nk columns (wk), each over the token's whole slice, eps_qk; the
+    remaining columns (v) pass through.  FlashNorm, abstract (norm then
+    linear) followed by layerwise QK-Norm (SwiftQK, abstract): [M, N]."""
+    W = as_f64(W)
+    N = W.shape[1]
+    assert 0 < nq and 0 < nk and nq + nk <= N
+    u = norm_then_project(x, w_in, W, eps) if input_norm else as_f64(x) @ W  # library matmul as one step
+    y = u.copy()
+    y[:, :nq] = rmsnorm(np.ascontiguousarray(u[:, :nq]), wq, eps_qk)
+    y[:, nq:nq + nk] = rmsnorm(np.ascontiguousarray(u[:, nq:nq + nk]), wk, eps_qk)
+    return y
+
+
 def round_bf16_bits(v) -> np.ndarray:
     """Round-to-nearest-even of float64 values to bfloat16; returns uint16 bit patterns."""
     v = as_f64(v)

@@ -300,3 +300,69 @@ def test_rmsnorm_elimination_needs_the_second_norm():
     # without the second norm the row scale 1/rms(x) survives: catches an identity applied too widely
     x, w, W = rand(4, 16) * 5, rand(16), rand(16, 8)
     assert not np.allclose(oracle.norm_then_project(x, w, W, 0.0), x @ oracle.fold_weights(w, W))
+
+
+# --------------------------------------------------------------- QKV projection + QK-Norm
+
+
+def _brute_qkv(x, w_in, W, wq, wk, nq, nk, eps, eps_qk):
+    # written out element by element in pure Python: the definition, nothing shared
+    M, K = len(x), len(x[0])
+    N = len(W[0])
+    out = [[0.0] * N for _ in range(M)]
+    for m in range(M):
+        r = 1.0 / math.sqrt(sum(v * v for v in x[m]) / K + eps)
+        u = [sum(x[m][k] * r * w_in[k] * W[k][n] for k in range(K)) for n in range(N)]
+        for lo, hi, w in ((0, nq, wq), (nq, nq + nk, wk)):
+            s = sum(u[n] * u[n] for n in range(lo, hi))
+            inv = 1.0 / math.sqrt(s / (hi - lo) + eps_qk)
+            for n in range(lo, hi):
+                out[m][n] = u[n] * inv * w[n - lo]
+        for n in range(nq + nk, N):
+            out[m][n] = u[n]
+    return np.array(out)
+
+
+@pytest.mark.parametrize("eps,eps_qk", [(0.0, 0.0), (1e-6, 1e-6), (0.3, 0.05)])
+def test_qkv_qknorm_brute_force(eps, eps_qk):
+    x, w_in, W = rand(3, 5), rand(5), rand(5, 11)
+    wq, wk = rand(4), rand(3)
+    got = oracle.qkv_proj_qknorm(x, w_in, W, wq, wk, 4, 3, eps, eps_qk)
+    ref = _brute_qkv(x.tolist(), w_in.tolist(), W.tolist(), wq.tolist(), wk.tolist(), 4, 3, eps, eps_qk)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_qkv_qknorm_identity_projection_reduces_to_rmsnorm():
+    # W = I, w_in = 1, eps = eps_qk = 0: the input norm only scales each row by a positive
+    # factor, which QK-Norm removes, so q and k are plain RMSNorms of x's own slices and v
+    # is the slice of RMSNorm(x)
+    nq, nk, nv = 6, 4, 5
+    d = nq + nk + nv
+    x, wq, wk = rand(7, d), rand(nq), rand(nk)
+    y = oracle.qkv_proj_qknorm(x, np.ones(d), np.eye(d), wq, wk, nq, nk, 0.0, 0.0)
+    np.testing.assert_allclose(y[:, :nq], oracle.rmsnorm(x[:, :nq].copy(), wq, 0.0), rtol=1e-12)
+    np.testing.assert_allclose(y[:, nq:nq + nk], oracle.rmsnorm(x[:, nq:nq + nk].copy(), wk, 0.0), rtol=1e-12)
+    np.testing.assert_allclose(y[:, nq + nk:], oracle.rmsnorm(x, np.ones(d), 0.0)[:, nq + nk:], rtol=1e-12)
+
+
+def test_qkv_qknorm_unit_rms_and_section_swap():
+    x, w_in, W = rand(5, 16), rand(16), rand(16, 20)
+    nq, nk = 8, 6
+    y = oracle.qkv_proj_qknorm(x, w_in, W, np.ones(nq), np.ones(nk), nq, nk, 1e-6, 0.0)
+    np.testing.assert_allclose(np.sqrt((y[:, :nq] ** 2).mean(1)), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(np.sqrt((y[:, nq:nq + nk] ** 2).mean(1)), 1.0, rtol=1e-12)
+    # moving k's columns in front of q's (with their weights) moves the outputs the same way
+    wq, wk = rand(nq), rand(nk)
+    a = oracle.qkv_proj_qknorm(x, w_in, W, wq, wk, nq, nk, 1e-6, 1e-3)
+    perm = np.r_[nq:nq + nk, 0:nq, nq + nk:20]
+    b = oracle.qkv_proj_qknorm(x, w_in, W[:, perm], wk, wq, nk, nq, 1e-6, 1e-3)
+    np.testing.assert_allclose(b, a[:, perm], rtol=1e-12, atol=1e-14)
+
+
+def test_qkv_qknorm_without_input_norm_is_scale_free_on_q_and_k():
+    # input_norm=False uses x as it is; q and k are still normalised, so scaling x changes only v
+    x, W = rand(4, 12), rand(12, 14)
+    a = oracle.qkv_proj_qknorm(x, None, W, np.ones(6), np.ones(4), 6, 4, 0.0, 0.0, input_norm=False)
+    b = oracle.qkv_proj_qknorm(3 * x, None, W, np.ones(6), np.ones(4), 6, 4, 0.0, 0.0, input_norm=False)
+    np.testing.assert_allclose(b[:, :10], a[:, :10], rtol=1e-12)
+    np.testing.assert_allclose(b[:, 10:], 3 * a[:, 10:], rtol=1e-12)

@@ -53,7 +53,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=None, help="timed steps (default depends on workload)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=QK_DEFAULT,
-                    choices=["tiny", "decode", "prefill_gqa", "long_context", "flashnorm_proj"])
+                    choices=["tiny", "decode", "prefill_gqa", "long_context", "flashnorm_proj",
+                             "qkv_proj_qknorm"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--strong", action="store_true",
@@ -251,6 +252,27 @@ def cpu_baseline_flashnorm(inp_host, budget_s: float):
                       f"[4096 x 12288] projection, fp64 C oracle, {elapsed:.1f} s of CPU work"}
 
 
+def cpu_baseline_qkv(inp_host, nq, nk, wq, wk, budget_s: float):
+    import oracle
+    x, w, Wm, eps = inp_host["x"], inp_host["w"], inp_host["W"], inp_host["eps"]
+    M = x.shape[0]
+    w64, W64, wq64, wk64 = oracle.as_f64(w), oracle.as_f64(Wm), oracle.as_f64(wq), oracle.as_f64(wk)
+    done, elapsed, chunk, pos = 0, 0.0, 8, 0
+    while elapsed < budget_s:
+        n = min(chunk, M - pos)
+        x64 = oracle.as_f64(x[pos:pos + n])
+        t0 = time.perf_counter()
+        oracle.qkv_proj_qknorm(x64, w64, W64, wq64, wk64, nq, nk, eps, eps)
+        elapsed += time.perf_counter() - t0
+        done += n
+        pos = (pos + n) % M
+        if elapsed < budget_s / 8:
+            chunk = min(M, chunk * 2)
+    return {"value": done / elapsed, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{done} rows of x (cycling over {M} rows) through RMSNorm, the [4096 x 12288] "
+                      f"projection and QK-Norm of q and k, fp64 C oracle, {elapsed:.1f} s of CPU work"}
+
+
 # ------------------------------------------------------------------------ reference arm
 
 
@@ -261,7 +283,15 @@ def run_reference(args):
     import torch
     from rmsnorm_qknorm_b200 import workloads as W
     steps = args.steps if args.steps is not None else 5
-    if args.workload == "flashnorm_proj":
+    if args.workload == "qkv_proj_qknorm":
+        wl = W.FLASHNORM_WORKLOAD
+        inp = W.make_flashnorm_inputs(seed=0, M=64)
+        nq = nk = wl.N // 3
+        wq, wk = W.make_qkv_norm_weights(nq, nk)
+        fn = lambda: cpu_baseline_qkv(inp, nq, nk, wq, wk, 4.0)  # noqa: E731
+        metric = "RMSNorm + QKV projection + QK-Norm tokens/s (fp64 CPU oracle)"
+        cfg = {"workload": "qkv_proj_qknorm", "M": wl.M, "K": wl.K, "nq": nq, "nk": nk, "nv": wl.N - 2 * nq}
+    elif args.workload == "flashnorm_proj":
         wl = W.FLASHNORM_WORKLOAD
         inp = W.make_flashnorm_inputs(seed=0, M=64)
         fn = lambda: cpu_baseline_flashnorm(inp, 4.0)  # noqa: E731
@@ -548,6 +578,131 @@ def run_flashnorm(args, rank, world, local, pg):
         }), flush=True)
 
 
+def run_qkv(args, rank, world, local, pg):
+    """RMSNorm -> QKV projection -> QK-Norm of q and k, x [8192, 4096], W [4096, 12288] = q | k | v."""
+    import torch
+    import rmsnorm_qknorm_b200 as qk
+    from rmsnorm_qknorm_b200 import workloads as W
+    from rmsnorm_qknorm_b200 import dist as qdist
+    qk.load_library()
+    wl = W.FLASHNORM_WORKLOAD
+    nq = nk = wl.N // 3
+    nv = wl.N - nq - nk
+    steps = args.steps if args.steps is not None else 200
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    inp = W.make_flashnorm_inputs(seed=qdist.rank_seed(0, rank), device=dev)
+    x, w, Wm = inp["x"], inp["w"], inp["W"]
+    wq, wk = W.make_qkv_norm_weights(nq, nk, device=dev)
+    Wf = qk.flashnorm_fold_weights(w, Wm)
+    y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
+    inv = torch.empty(wl.M, dtype=torch.float32, device=dev)
+    ws = torch.empty(qk.qkv_proj_qknorm_workspace_bytes(wl.M, nq, nk, nv), dtype=torch.uint8, device=dev)
+
+    def step(_i):  # statistics pass + one fused GEMM (q, k normalised in its epilogue)
+        qk.qkv_proj_qknorm(x, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms_out=inv, workspace=ws, out=y)
+
+    def gemm_only(_i):  # the fused GEMM alone (plus its 2 KB counter reset)
+        qk.qkv_proj_qknorm(x, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms=inv, workspace=ws, out=y)
+
+    def two_step(_i):  # our projection, then qknorm_fused on the q and k column blocks in place
+        qk.flashnorm_proj(x, Wf, wl.eps, inv_rms_out=inv, out=y)
+        qk.qknorm_fused(y[:, :nq], y[:, nq:nq + nk], wq, wk, wl.eps, 1, inplace=True)
+
+    xn = torch.empty_like(x)
+
+    def unfused(_i):  # RMSNorm kernel, cuBLAS with the original W, QK-Norm kernel
+        qk.qknorm_fused(x, None, w, None, wl.eps, 1, q_out=xn)
+        torch.matmul(xn, Wm, out=y)
+        qk.qknorm_fused(y[:, :nq], y[:, nq:nq + nk], wq, wk, wl.eps, 1, inplace=True)
+
+    for i in range(max(args.warmup, 3)):
+        for f in (step, gemm_only, two_step, unfused):
+            f(i)
+    barrier(pg)
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+        clocks.mark(True)
+    rounds = 5
+    per = max(steps // rounds, 1)
+    tot = {"step": 0.0, "two_step": 0.0, "unfused": 0.0}
+    gemm_ms = []
+    for _ in range(rounds):  # alternating rounds: every form sees the same clocks
+        tot["step"] += time_launches(step, per, stream)[0]
+        gemm_ms += time_launches(gemm_only, per, stream)[1]
+        tot["two_step"] += time_launches(two_step, per, stream)[0]
+        tot["unfused"] += time_launches(unfused, per, stream)[0]
+    steps = per * rounds
+    if clocks:
+        clocks.mark(False)
+    barrier(pg)
+    for key in tot:
+        tot[key] = max_over_ranks(tot[key], pg)
+    avg_gemm = max_over_ranks(statistics.mean(gemm_ms), pg)
+    clk = clocks.stop(gpu_index=local) if clocks else None
+    ms_per_step = tot["step"] / steps
+    value = world * wl.M / (ms_per_step * 1e-3)
+    pk, pk_kind = peaks()
+    tflops = wl.flops() / (avg_gemm * 1e-3) / 1e12
+    src = ["rmsnorm_qknorm_b200/csrc/qkv_qknorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
+           "rmsnorm_qknorm_b200/csrc/qkn_common.cuh", "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
+
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = x.cpu().pin_memory()
+        hy = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
+        dx = torch.empty_like(x)
+
+        def e2e_step(_i):
+            dx.copy_(hx, non_blocking=True)
+            qk.qkv_proj_qknorm(dx, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms_out=inv, workspace=ws, out=y)
+            hy.copy_(y, non_blocking=True)
+
+        e2e_step(0)
+        barrier(pg)
+        e_ms, _ = time_launches(e2e_step, args.e2e_steps, stream)
+        barrier(pg)
+        e_ms = max_over_ranks(e_ms, pg)
+        e2e = {"value": world * wl.M / (e_ms / args.e2e_steps * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2,
+               "note": "pinned host x -> device, qkv_proj_qknorm, device -> pinned host y, per step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = W.make_flashnorm_inputs(seed=0, device="cpu", M=256)
+        hwq, hwk = W.make_qkv_norm_weights(nq, nk)
+        cpu = cpu_baseline_qkv(host, nq, nk, hwq, hwk, args.cpu_seconds)
+
+    if rank == 0:
+        print(json.dumps({
+            "metric": "RMSNorm + QKV projection + QK-Norm tokens/s and tensor-core TFLOP/s (% of bf16 peak) "
+                      "on 1 GPU",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "qkv_proj_qknorm", "M": wl.M, "K": wl.K, "nq": nq, "nk": nk, "nv": nv,
+                       "eps": wl.eps, "parallelism": f"dp{world} (token batches, no collective)",
+                       "l2": "inputs larger than L2 (x 67 MB + W' 101 MB)"},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / pk["bf16_tflops"], "kernel": "qkv_qknorm_gemm_kernel",
+                         "traffic": traffic_for("qkv_qknorm_gemm_kernel", "qkv_proj_qknorm", src),
+                         "avg_launch_us": avg_gemm * 1e3, "flops_per_launch": wl.flops(),
+                         "launch_timing": "CUDA events around each call with a given 1/rms (counter reset + "
+                                          "the fused GEMM)",
+                         "peak_source": f"{pk_kind} cuBLAS bf16 burst"},
+            "comparison": {"fused_ms_per_step": ms_per_step,
+                           "two_step_ms_per_step": tot["two_step"] / steps,
+                           "unfused_ms_per_step": tot["unfused"] / steps,
+                           "speedup_vs_two_step": tot["two_step"] / tot["step"],
+                           "speedup_vs_unfused": tot["unfused"] / tot["step"],
+                           "two_step": "flashnorm_proj then qknorm_fused on q and k in place",
+                           "unfused": "qknorm_fused RMSNorm writing x_hat, torch.matmul (cuBLAS) with W, "
+                                      "qknorm_fused on q and k"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * steps, "clocks": clk,
+        }), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -556,6 +711,8 @@ def main():
     try:
         if args.workload == "flashnorm_proj":
             run_flashnorm(args, rank, world, local, pg)
+        elif args.workload == "qkv_proj_qknorm":
+            run_qkv(args, rank, world, local, pg)
         else:
             run_qknorm(args, rank, world, local, pg)
     finally:

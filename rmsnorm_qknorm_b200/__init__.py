@@ -33,6 +33,9 @@ __all__ = [
     "load_library",
     "library_path",
     "qknorm_fused",
+    "qknorm_fused_host",
+    "qkv_proj_qknorm",
+    "qkv_proj_qknorm_workspace_bytes",
     "rmsnorm_partial_stats",
     "flashnorm_fold_weights",
     "flashnorm_proj",
@@ -90,8 +93,12 @@ def load_library() -> ctypes.CDLL:
         lib.qkv_norm_proj.argtypes = [p, p, p, i64, i64, i64, i64, i64, p, p, p, i32, f32, i32, p]
         lib.qknorm_fused_host.argtypes = [p, p, p, p, p, p, i64, i64, i64, i32, i32, f32, i32,
                                           p, ctypes.c_size_t, p]
+        lib.qkv_proj_qknorm.argtypes = [p, p, p, i64, i64, i64, i64, i64, p, p, i32, f32, f32, p, p,
+                                        p, ctypes.c_size_t, p]
+        lib.qkv_proj_qknorm_workspace_bytes.argtypes = [i64, i64, i64, i64]
+        lib.qkv_proj_qknorm_workspace_bytes.restype = ctypes.c_size_t
         lib.qkn_check_device.argtypes = [p]
-        for f in ("qknorm_fused", "qknorm_fused_host", "rmsnorm_partial_stats", "flashnorm_fold_weights",
+        for f in ("qknorm_fused", "qknorm_fused_host", "qkv_proj_qknorm", "rmsnorm_partial_stats", "flashnorm_fold_weights",
                   "flashnorm_proj", "rmsnorm_apply_partials", "qkv_norm_proj", "qkn_check_device"):
             getattr(lib, f).restype = ctypes.c_int
         lib.qkn_last_error.restype = ctypes.c_char_p
@@ -378,4 +385,63 @@ def qkv_norm_proj(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, nv:
         wk.data_ptr(), wv.data_ptr() if (wv is not None and nv > 0) else None, _dtype_code(wq.dtype),
         float(eps), int(n_seg), _stream(stream))
     _check("qkv_norm_proj", st)
+    return out
+
+
+def qkv_proj_qknorm_workspace_bytes(M: int, nq: int, nk: int, nv: int) -> int:
+    """Device scratch qkv_proj_qknorm needs for these sizes (bytes)."""
+    return int(load_library().qkv_proj_qknorm_workspace_bytes(M, nq, nk, nv))
+
+
+def qkv_proj_qknorm(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, nv: int,
+                    wq: torch.Tensor, wk: torch.Tensor, eps: float = 1e-6, eps_qk: float | None = None, *,
+                    input_norm: bool = True, inv_rms: torch.Tensor | None = None,
+                    inv_rms_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """[q | k | v] = QK-Norm of RMSNorm(x) W in one GEMM (q, k normalised in the epilogue).
+
+    The input norm's weights are folded into ``W_folded`` ([nq+nk+nv, K],
+    from ``flashnorm_fold_weights``).  Its 1/rms comes from ``inv_rms`` when
+    given, else a statistics pass writes it to ``inv_rms_out`` (allocated when
+    ``input_norm`` and not given); ``input_norm=False`` uses x unscaled.
+    ``eps_qk`` defaults to ``eps``.  ``workspace`` (uint8 CUDA tensor of at
+    least ``qkv_proj_qknorm_workspace_bytes``) avoids an allocation inside
+    the call.
+    """
+    _cuda(x, "x")
+    _cuda(W_folded, "W_folded")
+    if x.dim() != 2 or not x.is_contiguous() or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a contiguous bf16 [M, K] tensor")
+    M, K = x.shape
+    N = nq + nk + nv
+    if tuple(W_folded.shape) != (N, K) or not W_folded.is_contiguous() or W_folded.dtype != torch.bfloat16:
+        raise ValueError(f"W_folded must be a contiguous bf16 [{N}, {K}] tensor")
+    _vec(wq, "wq", nq)
+    _vec(wk, "wk", nk)
+    if wk.dtype != wq.dtype:
+        raise ValueError("wk must have wq's dtype")
+    if inv_rms is not None:
+        _vec(inv_rms, "inv_rms", M)
+        if inv_rms.dtype != torch.float32:
+            raise ValueError("inv_rms must be fp32")
+    elif input_norm and inv_rms_out is None:
+        inv_rms_out = torch.empty(M, dtype=torch.float32, device=x.device)
+    if inv_rms_out is not None:
+        _vec(inv_rms_out, "inv_rms_out", M)
+        if inv_rms_out.dtype != torch.float32:
+            raise ValueError("inv_rms_out must be fp32")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _cuda(workspace, "workspace")
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = load_library().qkv_proj_qknorm(
+        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, K, nq, nk, nv,
+        wq.data_ptr(), wk.data_ptr(), _dtype_code(wq.dtype), float(eps),
+        float(eps if eps_qk is None else eps_qk),
+        inv_rms.data_ptr() if inv_rms is not None else None,
+        inv_rms_out.data_ptr() if (inv_rms is None and inv_rms_out is not None) else None,
+        ws_ptr, ws_bytes, _stream(stream))
+    _check("qkv_proj_qknorm", st)
     return out

@@ -124,7 +124,9 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
 
 // Whole warp: waits until *cnt >= target.  Every lane's own acquire load sees
 // the final count, so the partial sums published before the release adds are
-// visible to all lanes afterwards.  Returns false after wait_ns.
+// visible to all lanes afterwards.  Returns false after wait_ns, or as soon as
+// another wait of this launch has given up (so one failure costs one limit,
+// not one per tile).
 __device__ __noinline__ bool wait_count(const unsigned *cnt, unsigned target, uint64_t wait_ns) {
     if (__all_sync(0xffffffffu, ld_acquire(cnt) >= target)) return true;
     const uint64_t t0 = global_timer();
@@ -133,8 +135,9 @@ __device__ __noinline__ bool wait_count(const unsigned *cnt, unsigned target, ui
             __nanosleep(64);
             if (__all_sync(0xffffffffu, ld_acquire(cnt) >= target)) return true;
         }
-        const int late = (global_timer() - t0 > wait_ns) ? 1 : 0;
-        if (__shfl_sync(0xffffffffu, late, 0)) return false;
+        const int give_up =
+            (global_timer() - t0 > wait_ns || *static_cast<volatile int *>(&g_qkv_error) != 0) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
     }
 }
 

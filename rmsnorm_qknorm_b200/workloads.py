@@ -170,3 +170,15 @@ def make_flashnorm_inputs(seed: int = 0, device="cpu", M: int | None = None,
     bf = torch.bfloat16
     return {"x": x.to(bf).contiguous(), "w": w.to(bf).contiguous(),
             "W": W.to(bf).contiguous(), "eps": wl.eps}
+
+
+def make_qkv_norm_weights(nq: int, nk: int, seed: int = 0, device="cpu"):
+    """QK-Norm weights for the QKV projection workload: wq [nq], wk [nk] ~ N(1, 0.1) in bf16.
+
+    Drawn in that order from one generator, in fp32, then rounded to bf16.
+    """
+    g = _gen(seed + 1, device)
+    f32 = torch.float32
+    wq = 1.0 + 0.1 * torch.randn(nq, generator=g, device=device, dtype=f32)
+    wk = 1.0 + 0.1 * torch.randn(nk, generator=g, device=device, dtype=f32)
+    return wq.to(torch.bfloat16).contiguous(), wk.to(torch.bfloat16).contiguous()

@@ -188,3 +188,31 @@ def test_host_entry_validation(lib):
     assert "workspace" in lib.qkn_last_error().decode()
     assert h(ws=P + 16) == ALIGN               # workspace must be 256-byte aligned
     assert h(T=0, q=None, k=None, qo=None, ko=None, ws=None) == OK
+
+
+def test_qkv_proj_qknorm_validation(lib):
+    # (x, Wf, y, M, K, nq, nk, nv, wq, wk, wdt, eps, eps_qk, inv, inv_out, ws, ws_bytes, stream)
+    f = lib.qkv_proj_qknorm
+
+    def c(x=P, Wf=P, y=P, M=8, K=64, nq=64, nk=32, nv=32, wq=P, wk=P, wdt=BF16, eps=1e-6, eps_qk=1e-6,
+          inv=None, inv_out=None, ws=None, nbytes=0):
+        return f(x, Wf, y, M, K, nq, nk, nv, wq, wk, wdt, eps, eps_qk, inv, inv_out, ws, nbytes, None)
+
+    assert c(wk=None) == NULL
+    assert c(y=None) == NULL
+    assert c(M=0) == SHAPE
+    assert c(nq=0) == SHAPE
+    assert c(nv=-8) == SHAPE
+    assert c(K=60) == SHAPE
+    assert c(nk=36) == SHAPE
+    assert c(wdt=7) == DTYPE
+    assert c(eps_qk=-1.0) == EPS
+    assert c(eps=float("nan"), inv_out=P) == EPS    # eps is used by the statistics pass
+    assert c(x=P + 8) == ALIGN
+    assert c(wq=P + 4) == ALIGN
+    assert c(ws=P + 8, nbytes=1 << 20) == ALIGN
+    need = lib.qkv_proj_qknorm_workspace_bytes(8, 64, 32, 32)
+    assert need > 0
+    assert c(ws=P, nbytes=need - 1) == SHAPE
+    assert "workspace" in lib.qkn_last_error().decode()
+    assert lib.qkv_proj_qknorm_workspace_bytes(0, 64, 32, 32) == 0

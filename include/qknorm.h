@@ -336,6 +336,18 @@ QKN_API qkn_status qkn_check_device(void *stream);
  */
 QKN_API qkn_status qkn_testing_arm_wait_fault(uint64_t wait_ns);
 
+/*
+ * qkn_testing_arm_exchange_fault -- TESTING ONLY.  Arms, for this host
+ * thread's next qkv_proj_qknorm call, a wait limit of wait_ns
+ * (0 < wait_ns <= 2 s) and one epilogue warp that does not count itself in
+ * after publishing its first partial sums, so the exchange waits of that row
+ * block run out.  The kernel then records the
+ * failure, stops waiting, and returns; qkn_check_device reports
+ * QKN_ERR_TIMEOUT.  No GPU fault is involved.  QKN_ERR_SHAPE for a wait_ns
+ * out of range.
+ */
+QKN_API qkn_status qkn_testing_arm_exchange_fault(uint64_t wait_ns);
+
 /* Message describing the last nonzero status returned on this host thread. */
 QKN_API const char *qkn_last_error(void);
 

@@ -51,7 +51,7 @@ using gemm::UMMA_K;
 constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
-constexpr int GROUP_M = 8;  // row blocks walked together so concurrent tiles share W' panels in L2
+constexpr int GROUP_M = 64;  // row blocks walked together: W' is read from DRAM about once per 64 row blocks
 
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
@@ -69,6 +69,7 @@ struct Args {
     int w_f32;             // 1: fp32 QK-Norm weights, 0: bf16
     float eps;             // QK-Norm eps
     uint64_t wait_ns;      // limit of every wait
+    int skip_arrival;      // testing only: CTA 0's first epilogue warp does not count in on its first tile
 };
 
 struct Tile {
@@ -280,7 +281,8 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                 __threadfence();
                 __syncwarp();
                 unsigned *cnt = g.count + (t.m_blk * 2 + t.sec) * 4 + quarter;
-                if (lane == 0) red_release_add(cnt, 1u);
+                const bool skip = g.skip_arrival && blockIdx.x == 0 && it == 0 && quarter == 0;
+                if (lane == 0 && !skip) red_release_add(cnt, 1u);
                 const int ntiles = t.sec == 0 ? g.tq : g.tk;
                 if (!wait_count(cnt, (unsigned)ntiles, g.wait_ns) && lane == 0) atomicExch(&g_qkv_error, 1);
                 // fixed-order combine of the row's per-tile partial sums
@@ -356,6 +358,10 @@ Layout layout(int64_t M, int64_t nq, int64_t nk, int64_t nv) {
 }
 
 }  // namespace qkvn
+
+// Testing hook: the next qkv_proj_qknorm call on this host thread runs with
+// a short wait limit and one missing arrival (a count nothing completes).
+thread_local uint64_t t_exchange_fault_ns = 0;
 
 qkn_status read_qkv_error(int *flag) {
     cudaError_t e = cudaMemcpyFromSymbol(flag, g_qkv_error, sizeof(int));
@@ -464,6 +470,12 @@ extern "C" QKN_API qkn_status qkv_proj_qknorm(const void *x, const void *W_folde
         g.w_f32 = wdt == QKN_F32 ? 1 : 0;
         g.eps = eps_qk;
         g.wait_ns = kWaitTimeoutNs;
+        g.skip_arrival = 0;
+        if (t_exchange_fault_ns != 0) {  // one-shot test hook
+            g.wait_ns = t_exchange_fault_ns;
+            g.skip_arrival = 1;
+            t_exchange_fault_ns = 0;
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid, 1, 1);
         cfg.blockDim = dim3(qkvn::THREADS, 1, 1);
@@ -482,4 +494,12 @@ extern "C" QKN_API qkn_status qkv_proj_qknorm(const void *x, const void *W_folde
         if (e != cudaSuccess && st == QKN_OK) st = cuda_fail(e, "qkv_proj_qknorm: releasing the workspace");
     }
     return st;
+}
+
+extern "C" QKN_API qkn_status qkn_testing_arm_exchange_fault(uint64_t wait_ns) {
+    if (wait_ns == 0 || wait_ns > qkn::kWaitTimeoutNs)
+        return fail(QKN_ERR_SHAPE, "qkn_testing_arm_exchange_fault: wait_ns must be in (0, %llu]",
+                    (unsigned long long)qkn::kWaitTimeoutNs);
+    qkn::t_exchange_fault_ns = wait_ns;
+    return QKN_OK;
 }

@@ -216,3 +216,9 @@ def test_qkv_proj_qknorm_validation(lib):
     assert c(ws=P, nbytes=need - 1) == SHAPE
     assert "workspace" in lib.qkn_last_error().decode()
     assert lib.qkv_proj_qknorm_workspace_bytes(0, 64, 32, 32) == 0
+
+
+def test_exchange_fault_hook_validation(lib):
+    lib.qkn_testing_arm_exchange_fault.argtypes = [ctypes.c_uint64]
+    assert lib.qkn_testing_arm_exchange_fault(0) == SHAPE
+    assert lib.qkn_testing_arm_exchange_fault(3_000_000_000) == SHAPE

@@ -50,3 +50,33 @@ def test_wait_gives_up_and_reports_timeout(cuda_lib):
     assert lib.qkn_check_device(stream) == QKN_OK
     assert_bf16_close(qo, oracle.rmsnorm(inp["q"].cpu(), inp["wq"].cpu(), inp["eps"]), "after fault q")
     assert_bf16_close(ko, oracle.rmsnorm(inp["k"].cpu(), inp["wk"].cpu(), inp["eps"]), "after fault k")
+
+
+def test_exchange_wait_gives_up_and_reports_timeout(cuda_lib):
+    # the fused QKV kernel's cross-CTA exchange: one warp never counts itself in, so the
+    # waits of its row block's q section run out; the kernel records it and returns
+    lib = qk.load_library()
+    lib.qkn_testing_arm_exchange_fault.argtypes = [ctypes.c_uint64]
+    lib.qkn_testing_arm_exchange_fault.restype = ctypes.c_int
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.qkn_check_device(stream) == QKN_OK
+    M, K, nq, nk, nv = 512, 256, 1024, 512, 256
+    inp = W.make_flashnorm_inputs(seed=2, device="cuda", M=M, K=K, N=nq + nk + nv)
+    wq, wk = W.make_qkv_norm_weights(nq, nk, device="cuda")
+    Wf = qk.flashnorm_fold_weights(inp["w"], inp["W"])
+    assert lib.qkn_testing_arm_exchange_fault(50_000_000) == QKN_OK  # 50 ms limit
+    t0 = time.time()
+    qk.qkv_proj_qknorm(inp["x"], Wf, nq, nk, nv, wq, wk, inp["eps"])
+    st = lib.qkn_check_device(stream)
+    elapsed = time.time() - t0
+    assert st == QKN_ERR_TIMEOUT, lib.qkn_last_error()
+    assert b"fused QKV 1" in lib.qkn_last_error()
+    assert elapsed < 10.0
+    assert lib.qkn_check_device(stream) == QKN_OK  # cleared
+    # the next call on the same context is normal and correct
+    y = qk.qkv_proj_qknorm(inp["x"], Wf, nq, nk, nv, wq, wk, inp["eps"])
+    assert lib.qkn_check_device(stream) == QKN_OK
+    ref = oracle.qkv_proj_qknorm(inp["x"].cpu(), inp["w"].cpu(), inp["W"].cpu(), wq.cpu(), wk.cpu(), nq, nk,
+                                 inp["eps"], inp["eps"])
+    yd = y.cpu().double().numpy()
+    assert float(((yd - ref) ** 2).sum() ** 0.5 / (ref ** 2).sum() ** 0.5) <= 1e-2

@@ -500,11 +500,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
     float *scratch = reinterpret_cast<float *>(full + a.stages);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    // Programmatic dependent launch: the next kernel on the stream may be
+    // scheduled now (its blocks land on SMs as this grid's blocks exit), and
+    // this grid touches no global memory until the previous grid has finished
+    // and its writes are visible (a no-op when launched without the attribute).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.stages; ++s) mbar_init(smem_u32(&full[s]), 1);  // issuing lane + bytes
         mbar_init_fence();
     }
     __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // The first batch of weight loads goes out before the tile copies, so it
     // does not queue behind them in the memory system; the weights are
@@ -779,7 +785,20 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
         if (dev >= 0 && dev < 64) attr_bytes[dev] = smem;
     }
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
-    staged::rownorm_staged_kernel<TA, TW, STATS><<<(unsigned)grid, 32 * a.warps, smem, s>>>(a);
+    // launched with programmatic stream serialisation, so back-to-back
+    // launches overlap one grid's launch and setup with the previous one's tail
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(32 * a.warps, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, staged::rownorm_staged_kernel<TA, TW, STATS>, a);
+    if (e != cudaSuccess) return cuda_fail(e, "rownorm_staged_kernel launch");
     return check_launch("rownorm_staged_kernel launch");
 }
 

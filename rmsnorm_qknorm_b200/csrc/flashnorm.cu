@@ -72,6 +72,9 @@ __global__ void __launch_bounds__(256) inv_rms_kernel(const __nv_bfloat16 *__res
                                                       float *__restrict__ inv, int64_t M, int64_t K,
                                                       float eps) {
     constexpr int U = 8;
+    // let the projection that follows launch now: it streams x and W' through
+    // its MMAs while this pass runs, and only its epilogue waits for inv
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= M) return;  // whole warp leaves together
@@ -232,6 +235,11 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
         }
     } else if (warp < 6) {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
+        // Launched right behind the statistics pass (programmatic dependent
+        // launch), only these warps wait for that pass to finish and its 1/rms
+        // to be visible; the loads and MMAs above never read its output.  A
+        // no-op when the kernel was launched normally.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         const int quarter = warp & 3;  // TMEM lanes this warp may access: 32 * quarter ...
         int it = 0;
         for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++it) {
@@ -820,10 +828,12 @@ qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float 
 
 // inv == nullptr (and not unit_scale): the single-CTA kernel computes every
 // row's 1/rms itself (eps) and, when inv_out is given, stores it there.
-// The CTA-pair kernel serves every form; the single-CTA kernel is the
-// fallback when a two-CTA cluster cannot be launched on the device.
+// after_stats: the launch just before on `s` is this library's statistics
+// pass writing `inv` (and nothing the projection reads before its epilogue),
+// so the projection is launched as its programmatic dependent and overlaps it.
+// With QKN_GEMM_PAIR the CTA-pair kernel is tried first (never overlapped).
 qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
-                       float eps, float *inv_out, cudaStream_t s, bool unit_scale = false) {
+                       float eps, float *inv_out, cudaStream_t s, bool unit_scale = false, bool after_stats = false) {
     if (QKN_GEMM_PAIR && sm_count() >= 2) {
         const qkn_status st = launch_gemm_pair(x, Wf, y, inv, M, N, K, unit_scale, eps, inv_out, s);
         if (st != QKN_ERR_CUDA) return st;  // a launch the device refused falls through
@@ -855,7 +865,22 @@ qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv,
         attr_set[dev] = true;
     }
     const int grid = g.num_tiles < sm_count() ? g.num_tiles : sm_count();
-    gemm::flashnorm_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tx, tw, g);
+    if (after_stats) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
+        cfg.stream = s;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm::flashnorm_gemm_kernel, tx, tw, g);
+        if (e != cudaSuccess) return cuda_fail(e, "flashnorm_gemm_kernel launch");
+    } else {
+        gemm::flashnorm_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tx, tw, g);
+    }
     return check_launch("flashnorm_gemm_kernel launch");
 }
 
@@ -916,7 +941,9 @@ extern "C" QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded
         // the caller's buffer is the workspace of a separate row-statistics
         // pass, which leaves the matmul's shared-memory bandwidth to the MMA
         if (qkn_status st = launch_inv_rms(x, inv_rms_out, M, K, eps, s)) return st;
-        inv_rms = inv_rms_out;
+        // FlashNorm's "RMS and matmul in parallel": the projection starts while
+        // the statistics pass runs and waits for it only in its epilogue
+        return launch_gemm(x, W_folded, y, inv_rms_out, M, N, K, eps, nullptr, s, false, true);
     }
     // with no 1/rms at all the GEMM computes it beside the matmul (no workspace)
     return launch_gemm(x, W_folded, y, inv_rms, M, N, K, eps, nullptr, s);

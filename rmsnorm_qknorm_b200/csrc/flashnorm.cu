@@ -419,51 +419,6 @@ __device__ __forceinline__ void tile_coords(int tile, const Args &g, int &pm, in
     n = in_group / rows_in_group;
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Address of the same shared-memory object in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// try_wait with cluster-scope acquire: for phases completed by the peer CTA.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int *err) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = global_timer();
-    while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (global_timer() - t0 > kWaitTimeoutNs) {
-            atomicExch(err, 1);
-            return false;
-        }
-    }
-}
-
-// Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 // 2-D tensor copy into this CTA's shared memory whose bytes complete on the
 // barrier at `bar_cluster` (the even CTA's), for a CTA-pair MMA.  No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,

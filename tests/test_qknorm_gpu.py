@@ -106,10 +106,11 @@ def test_n_seg(cuda_lib, n_seg, dtype):
 # ------------------------------------------------------------- shapes and layouts
 
 
-@pytest.mark.parametrize("d", [1, 3, 8, 24, 100, 520, 1000, 4104, 65536, 65544, 131072])
+@pytest.mark.parametrize("d", [1, 3, 8, 24, 100, 520, 1000, 4104, 65536, 65544, 131072, 131080])
 def test_widths(cuda_lib, d):
     # odd widths and widths not a multiple of 8 take the element-wise kernel;
-    # 65536 bf16 is the widest row of the vector kernel, 131072 the element-wise one
+    # 65536 bf16 is the widest row one CTA holds, 65544 .. 131072 spread over a
+    # cluster of CTAs, and 131080 is past the cluster path (element-wise again)
     T = 3 if d >= 65536 else 19
     g = torch.Generator().manual_seed(d)
     x = torch.randn(T, d, generator=g).to(torch.bfloat16).to(DEV)

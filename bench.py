@@ -570,7 +570,8 @@ def run_flashnorm(args, rank, world, local, pg):
                          "frac": tflops / pk["bf16_tflops"], "kernel": "flashnorm_gemm_kernel",
                          "traffic": traffic_for("flashnorm_gemm_kernel", wl.name, src),
                          "avg_launch_us": avg_gemm * 1e3, "flops_per_launch": wl.flops(),
-                         "peak_source": f"{pk_kind} cuBLAS bf16 burst"},
+                         "peak_source": f"{pk_kind} cuBLAS bf16 burst",
+                         "frac_of_sustained": tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])},
             "comparison": {"unfused_ms_per_step": unf_ms / steps, "fused_ms_per_step": ms_per_step,
                            "speedup_vs_unfused": (unf_ms / steps) / ms_per_step,
                            "unfused": "qknorm_fused RMSNorm writing x_hat, then torch.matmul (cuBLAS) with W"},
@@ -690,7 +691,8 @@ def run_qkv(args, rank, world, local, pg):
                          "avg_launch_us": avg_gemm * 1e3, "flops_per_launch": wl.flops(),
                          "launch_timing": "CUDA events around each call with a given 1/rms (counter reset + "
                                           "the fused GEMM)",
-                         "peak_source": f"{pk_kind} cuBLAS bf16 burst"},
+                         "peak_source": f"{pk_kind} cuBLAS bf16 burst",
+                         "frac_of_sustained": tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])},
             "comparison": {"fused_ms_per_step": ms_per_step,
                            "two_step_ms_per_step": tot["two_step"] / steps,
                            "unfused_ms_per_step": tot["unfused"] / steps,

@@ -112,7 +112,8 @@ namespace gemm {
 constexpr int THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-7 row statistics
 constexpr int BAR_BYTES = 256;
 constexpr int INV_BYTES = 2 * BM * 4;                   // 1/rms of the rows of both accumulator tiles
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + INV_BYTES + 1024;  // + 1 KiB for alignment
+constexpr int EPI_BYTES = 4 * 2 * 2048;  // two 32x32 bf16 staging tiles per epilogue warp
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + INV_BYTES + 1024;  // + 1 KiB for alignment
 constexpr int GROUP_M = 16;  // tiles are walked in groups of 16 row blocks so concurrent tiles share operands in L2
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
@@ -144,15 +145,15 @@ __device__ __forceinline__ void tile_coords(int tile, const Args &g, int &m_blk,
 
 __global__ void __launch_bounds__(THREADS, 1)
 flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                      const Args g) {
+                      const __grid_constant__ CUtensorMap tmap_y, const Args g) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
     uint64_t *stats_full = bars + 2 * STAGES + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 6);
-    float *inv_buf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);  // [2][BM]
+    float *inv_buf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES);  // [2][BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -240,7 +241,14 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
         // to be visible; the loads and MMAs above never read its output.  A
         // no-op when the kernel was launched normally.
         asm volatile("griddepcontrol.wait;" ::: "memory");
+        // Each 32 x 32 block of y is staged in shared memory and written by one
+        // TMA store (whole lines, instead of 16 bytes to each of 32 rows).  The
+        // 64-byte swizzle puts a warp's 16-byte writes in the fewest wavefronts;
+        // a warp's two staging buffers alternate, and one is rewritten only
+        // after the store issued two blocks earlier has read it.
         const int quarter = warp & 3;  // TMEM lanes this warp may access: 32 * quarter ...
+        const uint32_t epi = smem_u32(smem + STAGES * STAGE_BYTES) + (uint32_t)quarter * 4096u;
+        int issued = 0;
         int it = 0;
         for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++it) {
             int m_blk, n_blk;
@@ -249,7 +257,8 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             const uint32_t acc_phase = (it >> 1) & 1;
             if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase, &g_device_error)) break;
             tc_fence_after();
-            const int row = m_blk * BM + quarter * 32 + lane;
+            const int row0 = m_blk * BM + quarter * 32;
+            const int row = row0 + lane;
             const bool row_ok = row < g.M;
             float r;
             if (g.unit_scale) {
@@ -260,32 +269,40 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             } else {
                 r = row_ok ? __ldg(g.inv_rms + row) : 0.f;
             }
-            __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld_32cols(tbase + c * 32, v);
                 const int col0 = n_blk * BN + c * 32;
-                if (row_ok) {
+                const uint32_t buf = epi + (uint32_t)(issued & 1) * 2048u;
+                if (lane == 0 && issued >= 2) bulk_wait_read1();  // the store that used this buffer has read it
+                __syncwarp();
+                const uint32_t rowaddr = buf + (uint32_t)lane * 64u;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int col = col0 + j * 8;
-                        if (col < g.N) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * r, __uint_as_float(v[8 * j + 1]) * r);
-                            o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * r, __uint_as_float(v[8 * j + 3]) * r);
-                            o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * r, __uint_as_float(v[8 * j + 5]) * r);
-                            o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * r, __uint_as_float(v[8 * j + 7]) * r);
-                            *reinterpret_cast<uint4 *>(yrow + col) = o;
-                        }
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    uint4 o;
+                    o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * r, __uint_as_float(v[8 * j + 1]) * r);
+                    o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * r, __uint_as_float(v[8 * j + 3]) * r);
+                    o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * r, __uint_as_float(v[8 * j + 5]) * r);
+                    o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * r, __uint_as_float(v[8 * j + 7]) * r);
+                    const uint32_t dst = rowaddr + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                 ::"r"(dst), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w) : "memory");
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (col0 < g.N && row0 < g.M) tma_store_2d(&tmap_y, buf, col0, row0);
+                    bulk_commit();
+                }
+                ++issued;
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
         }
+        if (lane == 0) bulk_wait_all();
     } else if (g.compute_inv) {
         // ---------------------------------------------------------------- row statistics (warps 6, 7)
         // FlashNorm's RMS runs beside the matmul: each x tile the TMA brings in
@@ -708,6 +725,20 @@ qkn_status make_tmap(CUtensorMap *m, const void *ptr, int64_t rows, int64_t inne
     return QKN_OK;
 }
 
+qkn_status make_tmap_store(CUtensorMap *m, void *ptr, int64_t rows, int64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return fail(QKN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(QKN_ERR_CUDA, "cuTensorMapEncodeTiled (y) failed (CUresult %d)", (int)r);
+    return QKN_OK;
+}
+
 qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float eps, cudaStream_t s) {
     const int64_t blocks = (M + 7) / 8;
     if (blocks > 0x7fffffffLL) return fail(QKN_ERR_SHAPE, "flashnorm_proj: M too large");
@@ -796,6 +827,8 @@ qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv,
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;
+    CUtensorMap ty;
+    if (qkn_status st = make_tmap_store(&ty, y, M, N)) return st;
     gemm::Args g;
     g.inv_rms = inv;
     g.inv_out = inv_out;
@@ -831,10 +864,10 @@ qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv,
         attr.val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm::flashnorm_gemm_kernel, tx, tw, g);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm::flashnorm_gemm_kernel, tx, tw, ty, g);
         if (e != cudaSuccess) return cuda_fail(e, "flashnorm_gemm_kernel launch");
     } else {
-        gemm::flashnorm_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tx, tw, g);
+        gemm::flashnorm_gemm_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tx, tw, ty, g);
     }
     return check_launch("flashnorm_gemm_kernel launch");
 }

@@ -81,6 +81,11 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
 // of 64 (inner) x box_rows, 128-byte swizzle, out-of-range elements read as 0.
 qkn_status make_tmap(CUtensorMap *m, const void *ptr, int64_t rows, int64_t inner, int box_rows);
 
+// 2-D bf16 tensor [rows][cols] as the destination of TMA stores: box of
+// 32 x 32, 64-byte swizzle (a 16-byte chunk j of staging row r sits at
+// position j ^ ((r >> 1) & 3)); parts of a box outside the tensor are skipped.
+qkn_status make_tmap_store(CUtensorMap *m, void *ptr, int64_t rows, int64_t cols);
+
 // inv[m] = 1/sqrt(sum_k x[m][k]^2 / K + eps) for bf16 x [M][K] (K a multiple
 // of 8, rows 16-byte aligned), on stream s.
 qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float eps, cudaStream_t s);

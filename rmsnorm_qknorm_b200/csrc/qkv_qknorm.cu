@@ -50,7 +50,8 @@ using gemm::UMMA_K;
 
 constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
+constexpr int EPI_BYTES = 4 * 2 * 2048;  // two 32x32 bf16 staging tiles per epilogue warp
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
 constexpr int GROUP_M = 64;  // row blocks walked together: W' is read from DRAM about once per 64 row blocks
 
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -158,10 +159,10 @@ __device__ __forceinline__ void load_w8(const void *w, int w_f32, int c, float (
 
 __global__ void __launch_bounds__(THREADS, 1)
 qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                       const Args g) {
+                       const __grid_constant__ CUtensorMap tmap_y, const Args g) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
@@ -244,6 +245,11 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         // ---------------------------------------------------------------- epilogue (warps 2..5)
         const int quarter = warp & 3;  // TMEM lanes 32 * quarter ... of the accumulator
         const int lrow = quarter * 32 + lane;
+        // 32 x 32 output blocks go out through shared memory and one TMA store
+        // each (two alternating staging buffers per warp, 64-byte swizzle); a
+        // block that a section ends inside is stored lane by lane instead
+        const uint32_t epi = smem_u32(smem + STAGES * STAGE_BYTES) + (uint32_t)quarter * 4096u;
+        int issued = 0;
         int it = 0;
         for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++it) {
             const Tile t = tile_of(tile, g);
@@ -294,39 +300,61 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                 w0 = t.col0 - (t.sec == 0 ? 0 : g.nq);
             }
             // pass 2: y = ((r * acc) * inv_qk) * w for q and k, r * acc for v; bf16 out
+            const int row0 = t.m_blk * BM + quarter * 32;
             __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
 #pragma unroll 1
             for (int c = 0; c < nchunks; ++c) {
                 uint32_t v[32];
                 gemm::tmem_ld_32cols(tbase + c * 32, v);
-                if (row_ok) {
+                const int base = c * 32;
+                const bool whole = base + 32 <= ncols;  // the same for the whole warp
+                const uint32_t buf = epi + (uint32_t)(issued & 1) * 2048u;
+                if (whole) {
+                    if (lane == 0 && issued >= 2) bulk_wait_read1();  // the store two blocks back has read it
+                    __syncwarp();
+                }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int off = c * 32 + j * 8;
-                        if (off < ncols) {
-                            float f[8];
+                for (int j = 0; j < 4; ++j) {
+                    const int off = base + j * 8;
+                    if (whole || (row_ok && off < ncols)) {
+                        float f[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * j + e]) * r;
-                            if (t.sec < 2) {
-                                float wv[8];
-                                load_w8(w, g.w_f32, w0 + off, wv);
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * j + e]) * r;
+                        if (t.sec < 2) {
+                            float wv[8];
+                            load_w8(w, g.w_f32, w0 + off, wv);
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) f[e] = (f[e] * inv_qk) * wv[e];
-                            }
-                            uint4 o;
-                            o.x = pack_bf16x2(f[0], f[1]);
-                            o.y = pack_bf16x2(f[2], f[3]);
-                            o.z = pack_bf16x2(f[4], f[5]);
-                            o.w = pack_bf16x2(f[6], f[7]);
+                            for (int e = 0; e < 8; ++e) f[e] = (f[e] * inv_qk) * wv[e];
+                        }
+                        uint4 o;
+                        o.x = pack_bf16x2(f[0], f[1]);
+                        o.y = pack_bf16x2(f[2], f[3]);
+                        o.z = pack_bf16x2(f[4], f[5]);
+                        o.w = pack_bf16x2(f[6], f[7]);
+                        if (whole) {
+                            const uint32_t dst = buf + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                         ::"r"(dst), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w) : "memory");
+                        } else {
                             *reinterpret_cast<uint4 *>(yrow + t.col0 + off) = o;
                         }
                     }
+                }
+                if (whole) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (row0 < g.M) tma_store_2d(&tmap_y, buf, t.col0 + base, row0);
+                        bulk_commit();
+                    }
+                    ++issued;
                 }
             }
             gemm::tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
         }
+        if (lane == 0) bulk_wait_all();
     }
 
     gemm::tc_fence_before();
@@ -432,6 +460,8 @@ extern "C" QKN_API qkn_status qkv_proj_qknorm(const void *x, const void *W_folde
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, W_folded, N, K, gemm::BN)) return st;
+    CUtensorMap ty;
+    if (qkn_status st = make_tmap_store(&ty, y, M, N)) return st;
 
     void *ws = workspace;
     bool owned = false;
@@ -486,7 +516,7 @@ extern "C" QKN_API qkn_status qkv_proj_qknorm(const void *x, const void *W_folde
         attr.val.cooperative = 1;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, qkvn::qkv_qknorm_gemm_kernel, tx, tw, g);
+        e = cudaLaunchKernelEx(&cfg, qkvn::qkv_qknorm_gemm_kernel, tx, tw, ty, g);
         if (e != cudaSuccess) st = cuda_fail(e, "qkv_qknorm_gemm_kernel launch");
     }
     if (owned) {

@@ -9,6 +9,7 @@
 // memory, and four epilogue warps read the accumulator back (tcgen05.ld),
 // multiply each row by its 1/rms and store bf16.  The 1/rms vector comes from
 // a small row-statistics kernel (or from the caller).
+#include <atomic>
 #include <cuda.h>
 #include <math.h>
 
@@ -696,14 +697,14 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {  // looked up once, thread-safe
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -774,19 +775,21 @@ qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float 
     g.compute_inv = (inv == nullptr && !unit_scale) ? 1 : 0;
     g.inv_out = g.compute_inv ? inv_out : nullptr;
     g.eps = eps;
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];  // per device: the attribute has been set
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const bool known = dev >= 0 && dev < 64;
+    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(gemm2::flashnorm_gemm_pair_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(flashnorm_gemm_pair_kernel)");
-        attr_set[dev] = true;
+        if (known) attr_set[dev].store(true, std::memory_order_release);
     }
     // a persistent grid must fit at once: as many pairs as the device can
     // keep resident together (two-SM clusters need both SMs of a pair free)
-    static int max_clusters[64] = {0};
-    if (dev >= 0 && dev < 64 && max_clusters[dev] == 0) {
+    static std::atomic<int> max_clusters[64];  // per device; 0 until measured
+    int pairs = known ? max_clusters[dev].load(std::memory_order_relaxed) : 0;
+    if (pairs == 0) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeClusterDimension;
@@ -804,9 +807,9 @@ qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float 
             cudaGetLastError();
             n = sm_count() / 2;
         }
-        max_clusters[dev] = n;
+        pairs = n;
+        if (known) max_clusters[dev].store(n, std::memory_order_relaxed);
     }
-    const int pairs = (dev >= 0 && dev < 64) ? max_clusters[dev] : sm_count() / 2;
     const int grid = 2 * (g.num_tiles < pairs ? g.num_tiles : pairs);
     gemm2::flashnorm_gemm_pair_kernel<<<grid, gemm2::THREADS, gemm2::SMEM_BYTES, s>>>(tx, tw, g);
     return check_launch("flashnorm_gemm_pair_kernel launch");
@@ -843,14 +846,15 @@ qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv,
     g.n_blocks = (int)((N + gemm::BN - 1) / gemm::BN);
     g.k_blocks = (int)((K + gemm::BK - 1) / gemm::BK);
     g.num_tiles = g.m_blocks * g.n_blocks;
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];  // per device: the attribute has been set
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const bool known = dev >= 0 && dev < 64;
+    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(gemm::flashnorm_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              gemm::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(flashnorm_gemm_kernel)");
-        attr_set[dev] = true;
+        if (known) attr_set[dev].store(true, std::memory_order_release);
     }
     const int grid = g.num_tiles < sm_count() ? g.num_tiles : sm_count();
     if (after_stats) {

@@ -12,6 +12,7 @@
 // memory when a row spans several warps), then combined left to right -- the
 // on-chip analogue of the shards' scalar exchange.  Query rows and key rows
 // are two jobs of the same launch.
+#include <atomic>
 #include <math.h>
 
 #include <mutex>
@@ -899,19 +900,19 @@ qkn_status launch_cluster(const Tensor2 *ts, int njobs, int64_t rows, int n_seg,
         J.per_cta = (J.nchunks + C - 1) / C;
     }
     // as many clusters as rows, at most as many as are resident at once; each loops over rows
-    static int per_sm[64] = {};  // per instantiation and device
+    static std::atomic<int> per_sm[64];  // per instantiation and device; 0 until measured
     int dev = 0;
     cudaGetDevice(&dev);
-    int blocks_per_sm = 1;
-    if (dev >= 0 && dev < 64) {
-        int &cached = per_sm[dev];
-        if (cached == 0 &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cached, cl::rownorm_cluster_kernel<TA, TW, STATS>,
-                                                          cl::kBlock, 0) != cudaSuccess) {
+    const bool known = dev >= 0 && dev < 64;
+    int blocks_per_sm = known ? per_sm[dev].load(std::memory_order_relaxed) : 0;
+    if (blocks_per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, cl::rownorm_cluster_kernel<TA, TW, STATS>,
+                                                          cl::kBlock, 0) != cudaSuccess ||
+            blocks_per_sm <= 0) {
             cudaGetLastError();
-            cached = 1;
+            blocks_per_sm = 1;
         }
-        blocks_per_sm = cached > 0 ? cached : 1;
+        if (known) per_sm[dev].store(blocks_per_sm, std::memory_order_relaxed);
     }
     const int64_t total = rows * njobs;
     const int64_t fit = (int64_t)blocks_per_sm * sm_count() / C > 0 ? (int64_t)blocks_per_sm * sm_count() / C : 1;
@@ -1019,15 +1020,19 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
         a.total_tiles += J.ntiles;
     }
     const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes);
-    static int attr_bytes[64] = {0};
+    // the attribute is a cap: set once per device to the whole budget the
+    // geometry ever asks for
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || attr_bytes[dev] < smem) {
+    const bool known = dev >= 0 && dev < 64;
+    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(staged::rownorm_staged_kernel<TA, TW, STATS>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_STAGED_SMEM_LIMIT);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rownorm_staged_kernel)");
-        if (dev >= 0 && dev < 64) attr_bytes[dev] = smem;
+        if (known) attr_set[dev].store(true, std::memory_order_release);
     }
+    static_assert(QKN_STAGED_SMEM_LIMIT <= 227 * 1024, "the staged geometry's budget is a valid attribute");
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
     // launched with programmatic stream serialisation, so back-to-back
     // launches overlap one grid's launch and setup with the previous one's tail

@@ -24,6 +24,7 @@
 // tile with the lowest index therefore waits only for tiles that their CTAs
 // reach without waiting on anything later, and every wait ends.  Each wait is
 // also bounded in time and records a failure in g_qkv_error.
+#include <atomic>
 #include <cuda.h>
 #include <math.h>
 
@@ -443,14 +444,15 @@ extern "C" QKN_API qkn_status qkv_proj_qknorm(const void *x, const void *W_folde
                     (long long)nq, (long long)nk, grid);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];  // per device: the attribute has been set
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const bool known = dev >= 0 && dev < 64;
+    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(qkvn::qkv_qknorm_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              qkvn::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv_qknorm_gemm_kernel)");
-        attr_set[dev] = true;
+        if (known) attr_set[dev].store(true, std::memory_order_release);
     }
 
     if (inv_rms == nullptr && inv_rms_out != nullptr) {

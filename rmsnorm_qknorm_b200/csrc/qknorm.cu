@@ -245,6 +245,7 @@ struct Job {
     int d, row_bytes, nchunks, seg_chunks;
     int w_offset;        // byte offset of this job's fp32 weights in shared memory
     int rows_per_tile;
+    int narrow_cpl;      // 1, 2 or 4: a narrow row whose segments are whole lane groups; 0 otherwise
     int64_t ntiles;
 };
 
@@ -283,6 +284,7 @@ __device__ __forceinline__ Job pick(const Args &a, int which) {
     J.seg_chunks = which ? j1.seg_chunks : j0.seg_chunks;
     J.w_offset = which ? j1.w_offset : j0.w_offset;
     J.rows_per_tile = which ? j1.rows_per_tile : j0.rows_per_tile;
+    J.narrow_cpl = which ? j1.narrow_cpl : j0.narrow_cpl;
     J.ntiles = which ? j1.ntiles : j0.ntiles;
     return J;
 }
@@ -356,16 +358,17 @@ __device__ __forceinline__ void apply_chunk(const uint4 &v, int c, float2 inv2, 
     st_stream_batched(yr + (int64_t)c * 16, Pairs<TA>::put(p));
 }
 
-// One row held in shared memory, processed by one warp.  `part` is the warp's
-// [8][32] scratch for lane partials; `wsm` the job's fp32 weights.
+// Statistic of one row held in shared memory, by one warp (any width): lane
+// l adds its chunks l, l + 32, ... in order into a running pair sum that is
+// parked in the warp's [8][32] scratch `part` whenever a segment ends; the 8
+// slots are reduced over the warp by recursive halving (lanes 4j .. 4j+3 end
+// with segment j) and the segments added left to right.  Returns S.
 template <typename TA, bool STATS>
-__device__ __forceinline__ void process_row(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
-                                            int64_t row, int lane, float *part) {
+__device__ __forceinline__ float row_statistic(const Args &a, const Job &J, const uint8_t *srow, int64_t row,
+                                               int lane, float *part) {
     const int nchunks = J.nchunks;
     const int n_seg = a.n_seg;
     const int sc = J.seg_chunks;
-
-    // ---- statistic
 #pragma unroll
     for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
     float2 cur = make_float2(0.f, 0.f);
@@ -446,8 +449,66 @@ __device__ __forceinline__ void process_row(const Args &a, const Job &J, const u
     }
     __syncwarp();  // the scratch is rewritten by the next row
 
+    return S;
+}
+
+// Statistic of a narrow row (32 * CPL chunks, CPL <= 4) whose segments are
+// whole groups of lanes: lane l sums its CPL contiguous chunks l*CPL ..
+// l*CPL + CPL - 1 (all in segment l / LPS, LPS = 32 / n_seg lanes per
+// segment), visiting them in an order rotated with the lane so a warp's
+// 16-byte shared-memory reads take the fewest wavefronts; then each segment
+// is reduced over its lanes (a fixed butterfly) and the segments are added
+// left to right.  Nothing is parked: every lane stays inside one segment.
+// Returns S; `seg` receives the lane's segment total.
+template <typename TA, int CPL>
+__device__ __forceinline__ float narrow_statistic(const uint8_t *srow, int lane, int n_seg, float &seg) {
+    constexpr int ROT = CPL == 4 ? 1 : 2;  // lanes that share a rotation step
+    float2 cur = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+        const int c = lane * CPL + ((u + (lane >> ROT)) & (CPL - 1));
+        cur = __fadd2_rn(cur, chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)));
+    }
+    float r = cur.x + cur.y;
+    const int lps = 32 / n_seg;
+    for (int off = 1; off < lps; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+    seg = r;
+    float tot[kFastMaxSeg];
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) tot[j] = __shfl_sync(0xffffffffu, r, (j * lps) & 31);
+    float S = 0.f;
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j)
+        if (j < n_seg) S += tot[j];
+    return S;
+}
+
+// One row held in shared memory, processed by one warp.  `part` is the warp's
+// [8][32] scratch for lane partials; `wsm` the job's fp32 weights.  NARROW:
+// the launch has narrow rows (the narrow statistic is compiled in; launches
+// without them keep the wide path alone, and its register budget).
+template <typename TA, bool STATS, bool NARROW>
+__device__ __forceinline__ void process_row(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
+                                            int64_t row, int lane, float *part) {
+    const int nchunks = J.nchunks;
+    float S;
+    if (NARROW && J.narrow_cpl != 0) {
+        const int n_seg = a.n_seg;
+        float seg;
+        if (J.narrow_cpl == 1) S = narrow_statistic<TA, 1>(srow, lane, n_seg, seg);
+        else if (J.narrow_cpl == 2) S = narrow_statistic<TA, 2>(srow, lane, n_seg, seg);
+        else S = narrow_statistic<TA, 4>(srow, lane, n_seg, seg);
+        if constexpr (STATS) {
+            const int lps = 32 / n_seg;
+            if ((lane & (lps - 1)) == 0) a.partial[row * n_seg + lane / lps] = seg;
+        }
+    } else {
+        S = row_statistic<TA, STATS>(a, J, srow, row, lane, part);
+    }
+
     // ---- apply
     if constexpr (!STATS) {
+        constexpr int G = 32 * kUnroll;  // chunks per group
         const float inv = rsqrtf(S / (float)J.d + a.eps);
         const float2 inv2 = make_float2(inv, inv);
         uint8_t *yr = J.y + row * J.ldo_bytes;
@@ -491,7 +552,7 @@ __device__ __forceinline__ void issue_tile(const Args &a, int64_t tile, int64_t 
         bulk_g2s(dst + r * J.row_bytes, J.x + (row0 + r) * J.ld_bytes, (uint32_t)J.row_bytes, fb);
 }
 
-template <typename TA, typename TW, bool STATS>
+template <typename TA, typename TW, bool STATS, bool NARROW>
 __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int W = a.warps, SB = a.stage_bytes;
@@ -609,7 +670,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
         const uint8_t *sbase = smem + (size_t)stage * SB;
         const float4 *wsm = reinterpret_cast<const float4 *>(wbase + J.w_offset);
         for (int r = 0; r < nrows; ++r)
-            process_row<TA, STATS>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
+            process_row<TA, STATS, NARROW>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
         __syncwarp();
         // refill this stage with the warp's tile k + spw
         const int64_t next = tile + spw * step;
@@ -979,6 +1040,39 @@ bool staged_geometry(int64_t max_row_bytes, int64_t w_bytes, int *warps, int *sp
 // next staged-kernel launch); see qkn_testing_arm_wait_fault.
 thread_local uint64_t t_fault_wait_ns = 0;
 
+// One instantiation of the staged kernel, launched with programmatic stream
+// serialisation, so back-to-back launches overlap one grid's launch and
+// setup with the previous one's tail.
+template <typename TA, typename TW, bool STATS, bool NARROW>
+qkn_status launch_staged_kernel(const staged::Args &a, int grid, int smem, cudaStream_t s) {
+    // the attribute is a cap: set once per device to the whole budget the
+    // geometry ever asks for
+    static std::atomic<bool> attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool known = dev >= 0 && dev < 64;
+    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
+        cudaError_t e = cudaFuncSetAttribute(staged::rownorm_staged_kernel<TA, TW, STATS, NARROW>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_STAGED_SMEM_LIMIT);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rownorm_staged_kernel)");
+        if (known) attr_set[dev].store(true, std::memory_order_release);
+    }
+    static_assert(QKN_STAGED_SMEM_LIMIT <= 227 * 1024, "the staged geometry's budget is a valid attribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(32 * a.warps, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, staged::rownorm_staged_kernel<TA, TW, STATS, NARROW>, a);
+    if (e != cudaSuccess) return cuda_fail(e, "rownorm_staged_kernel launch");
+    return check_launch("rownorm_staged_kernel launch");
+}
+
 template <typename TA, typename TW, bool STATS>
 qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps, float *partial,
                          int warps, int spw, int stage_bytes, cudaStream_t s) {
@@ -1016,39 +1110,21 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
         J.w_offset = a.w_bytes;
         if (!STATS) a.w_bytes += (int)(t.d * 4);
         J.rows_per_tile = stage_bytes / J.row_bytes;
+        // narrow rows of 32, 64 or 128 chunks whose segments are whole power-of-two lane groups
+        J.narrow_cpl = 0;
+        if (J.nchunks % 32 == 0 && J.nchunks <= 128) {
+            const int cpl = J.nchunks / 32, lps = 32 / n_seg;
+            if (lps * n_seg == 32 && (lps & (lps - 1)) == 0 && J.seg_chunks == cpl * lps) J.narrow_cpl = cpl;
+        }
         J.ntiles = (rows + J.rows_per_tile - 1) / J.rows_per_tile;
         a.total_tiles += J.ntiles;
     }
     const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes);
-    // the attribute is a cap: set once per device to the whole budget the
-    // geometry ever asks for
-    static std::atomic<bool> attr_set[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const bool known = dev >= 0 && dev < 64;
-    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(staged::rownorm_staged_kernel<TA, TW, STATS>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_STAGED_SMEM_LIMIT);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rownorm_staged_kernel)");
-        if (known) attr_set[dev].store(true, std::memory_order_release);
-    }
-    static_assert(QKN_STAGED_SMEM_LIMIT <= 227 * 1024, "the staged geometry's budget is a valid attribute");
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
-    // launched with programmatic stream serialisation, so back-to-back
-    // launches overlap one grid's launch and setup with the previous one's tail
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(32 * a.warps, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr.val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, staged::rownorm_staged_kernel<TA, TW, STATS>, a);
-    if (e != cudaSuccess) return cuda_fail(e, "rownorm_staged_kernel launch");
-    return check_launch("rownorm_staged_kernel launch");
+    bool narrow = false;
+    for (int i = 0; i < njobs; ++i) narrow = narrow || a.job[i].narrow_cpl != 0;
+    if (narrow) return launch_staged_kernel<TA, TW, STATS, true>(a, (int)grid, smem, s);
+    return launch_staged_kernel<TA, TW, STATS, false>(a, (int)grid, smem, s);
 }
 
 template <typename TA, typename TW, bool STATS>

@@ -233,3 +233,32 @@ def test_partial_stats_full_size_rows(cuda_lib):
         # the combined statistic of the partials is the full-row statistic
         full = oracle.segment_partials(inp[key].cpu(), 1)[:, 0]
         np.testing.assert_allclose(oracle.combine_partials(p.cpu().double().numpy()), full, rtol=1e-5)
+
+
+# --------------------------------------------------- narrow rows (lane-group segments)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("d,n_seg", [(256, 1), (256, 8), (512, 4), (512, 8), (1024, 2), (1024, 8), (1000, 8)])
+def test_narrow_rows(cuda_lib, dtype, d, n_seg):
+    # rows of 32, 64 or 128 16-byte chunks whose segments are whole lane groups take the
+    # narrow statistic (each lane sums contiguous chunks of one segment); 1000 does not
+    if dtype == torch.float32 and d == 1000:
+        pytest.skip("1000 fp32 elements: 250 chunks, not a narrow row")
+    T = 45
+    g = torch.Generator().manual_seed(d + n_seg)
+    x = (torch.randn(T, d, generator=g) * 2).to(dtype).to(DEV)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(dtype).to(DEV)
+    y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, n_seg)
+    # with a wide job beside it in the same launch (the prefill arrangement)
+    xw = torch.randn(T, 5120, generator=g).to(dtype).to(DEV)
+    ww = torch.ones(5120, dtype=dtype, device=DEV)
+    y2, y3 = qk.qknorm_fused(xw, x, ww, w, 1e-6, n_seg)
+    p = qk.rmsnorm_partial_stats(x, n_seg)
+    torch.cuda.synchronize()
+    check(y, x, w, 1e-6, f"narrow d={d} n_seg={n_seg}")
+    check(y3, x, w, 1e-6, f"narrow beside wide d={d} n_seg={n_seg}")
+    check(y2, xw, ww, 1e-6, "wide beside narrow")
+    assert torch.equal(y.view(torch.int16) if dtype == torch.bfloat16 else y,
+                       y3.view(torch.int16) if dtype == torch.bfloat16 else y3)
+    assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials d={d}")

@@ -831,33 +831,59 @@ __global__ void __launch_bounds__(kBlock) rownorm_cluster_kernel(const Args a) {
             const int c = c_lo + i * kBlock + (int)threadIdx.x;
             v[i] = c < c_hi ? ld_stream(xr + (int64_t)c * 16) : make_uint4(0u, 0u, 0u, 0u);
         }
-        // 2. sum of squares of every chunk
-#pragma unroll
-        for (int i = 0; i < kCpt; ++i) {
-            const int c = c_lo + i * kBlock + (int)threadIdx.x;
-            if (c < c_hi) {
-                float f[E];
-                Chunk<TA>::unpack(v[i], f);
-                float s = 0.f;
-#pragma unroll
-                for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
-                sq[c - c_lo] = s;
-            }
-        }
-        __syncthreads();
-        // 3. one partial per segment touched: lane l adds its contiguous share of
-        //    the piece's chunks in order, then a fixed butterfly over the warp
         const int j0 = c_lo < c_hi ? c_lo / J.seg_chunks : 0;
         const int npieces = c_lo < c_hi ? (c_hi - 1) / J.seg_chunks - j0 + 1 : 0;
-        for (int p = warp; p < npieces; p += kBlock / 32) {
-            const int j = j0 + p;
-            const int lo = max(c_lo, j * J.seg_chunks) - c_lo;
-            const int len = min(c_hi, (j + 1) * J.seg_chunks) - c_lo - lo;
-            const int b0 = lo + (lane * len) / 32, b1 = lo + ((lane + 1) * len) / 32;
-            float s = 0.f;
-            for (int k = b0; k < b1; ++k) s += sq[k];
-            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (lane == 0) piece[p] = s;
+        if (npieces == 1) {
+            // 2-3. the slice lies in one segment: each thread adds its chunks'
+            //      sums in order, a fixed butterfly per warp, the 8 warp sums in order
+            float t = 0.f;
+#pragma unroll
+            for (int i = 0; i < kCpt; ++i) {
+                const int c = c_lo + i * kBlock + (int)threadIdx.x;
+                if (c < c_hi) {
+                    float f[E];
+                    Chunk<TA>::unpack(v[i], f);
+                    float s = 0.f;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+                    t += s;
+                }
+            }
+            for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+            if (lane == 0) sq[warp] = t;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float s = 0.f;
+                for (int w = 0; w < kBlock / 32; ++w) s += sq[w];
+                piece[0] = s;
+            }
+        } else {
+            // 2. sum of squares of every chunk
+#pragma unroll
+            for (int i = 0; i < kCpt; ++i) {
+                const int c = c_lo + i * kBlock + (int)threadIdx.x;
+                if (c < c_hi) {
+                    float f[E];
+                    Chunk<TA>::unpack(v[i], f);
+                    float s = 0.f;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+                    sq[c - c_lo] = s;
+                }
+            }
+            __syncthreads();
+            // 3. one partial per segment touched: lane l adds its contiguous share of
+            //    the piece's chunks in order, then a fixed butterfly over the warp
+            for (int p = warp; p < npieces; p += kBlock / 32) {
+                const int j = j0 + p;
+                const int lo = max(c_lo, j * J.seg_chunks) - c_lo;
+                const int len = min(c_hi, (j + 1) * J.seg_chunks) - c_lo - lo;
+                const int b0 = lo + (lane * len) / 32, b1 = lo + ((lane + 1) * len) / 32;
+                float s = 0.f;
+                for (int k = b0; k < b1; ++k) s += sq[k];
+                for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+                if (lane == 0) piece[p] = s;
+            }
         }
         __syncthreads();
         const int buf = it & 1;

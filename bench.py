@@ -403,7 +403,8 @@ def run_qknorm(args, rank, world, local, pg):
     value = global_tokens / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
     achieved = per_set / (avg_launch_ms * 1e-3) / 1e9
-    src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
+    src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/rownorm_staged.cuh",
+           "rmsnorm_qknorm_b200/csrc/rownorm_register.cuh", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
            "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
     traffic = traffic_for("rownorm_staged_kernel", wl.name, src) if args.tokens is None else None
 

@@ -25,6 +25,12 @@ inline size_t dtype_size(qkn_dtype t) { return t == QKN_F32 ? 4 : 2; }
 
 inline bool valid_dtype(int t) { return t == QKN_F32 || t == QKN_BF16; }
 
+// n_seg within [1, QKN_MAX_SEG], else QKN_ERR_SHAPE with a message.
+inline qkn_status check_seg(int n_seg) {
+    if (n_seg < 1 || n_seg > QKN_MAX_SEG) return fail(QKN_ERR_SHAPE, "n_seg=%d outside [1, %d]", n_seg, QKN_MAX_SEG);
+    return QKN_OK;
+}
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

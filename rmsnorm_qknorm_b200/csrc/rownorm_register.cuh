@@ -1,0 +1,227 @@
+// Register-resident row kernels: the vectorised kernel (a row in the registers
+// of a group of threads) and the element-wise kernel for any alignment.
+//
+// Included by qknorm.cu only: the kernels are instantiated by its dispatch
+// and share its device error word g_norm_error (one translation unit).
+#pragma once
+
+#include "qkn_common.cuh"
+#include "qkn_sync.cuh"
+
+namespace qkn {
+
+constexpr int kFastMaxSeg = 8;    // segments handled by the vectorised kernel
+constexpr int kMaxWarps = 32;     // 1024-thread blocks at most
+
+// One set of rows to normalise (the query rows or the key rows).
+struct RowJob {
+    const uint8_t *x;     // row 0 of the input
+    uint8_t *y;           // row 0 of the output (may equal x: in place)
+    const void *w;        // weights [d]
+    int64_t ld_bytes;     // input row pitch in bytes
+    int64_t ldo_bytes;    // output row pitch in bytes
+    int64_t rows;
+    int d;                // row width in elements
+    int nchunks;          // d / elements-per-16-byte-chunk   (vector kernel)
+    int seg_chunks;       // chunks per segment               (vector kernel)
+    float inv_seg_chunks; // 1 / seg_chunks, for the segment index of a chunk
+    int tpr_log2;         // log2(threads per row)            (vector kernel)
+    int rows_per_cta;
+    int64_t nblocks;
+};
+
+struct RowArgs {
+    RowJob job[2];
+    int n_seg;
+    float eps;
+    float *partial;       // [rows][n_seg] output of the statistics-only mode
+};
+
+// Field-wise select of job 0 or 1 (keeps the kernel parameters in the
+// constant bank instead of copying the array to local memory).
+__device__ __forceinline__ RowJob pick_job(const RowArgs &a, int which) {
+    const RowJob &j0 = a.job[0], &j1 = a.job[1];
+    RowJob J;
+    J.x = which ? j1.x : j0.x;
+    J.y = which ? j1.y : j0.y;
+    J.w = which ? j1.w : j0.w;
+    J.ld_bytes = which ? j1.ld_bytes : j0.ld_bytes;
+    J.ldo_bytes = which ? j1.ldo_bytes : j0.ldo_bytes;
+    J.rows = which ? j1.rows : j0.rows;
+    J.d = which ? j1.d : j0.d;
+    J.nchunks = which ? j1.nchunks : j0.nchunks;
+    J.seg_chunks = which ? j1.seg_chunks : j0.seg_chunks;
+    J.inv_seg_chunks = which ? j1.inv_seg_chunks : j0.inv_seg_chunks;
+    J.tpr_log2 = which ? j1.tpr_log2 : j0.tpr_log2;
+    J.rows_per_cta = which ? j1.rows_per_cta : j0.rows_per_cta;
+    J.nblocks = which ? j1.nblocks : j0.nblocks;
+    return J;
+}
+
+// ---------------------------------------------------------------------------
+// Vectorised kernel: a row lives in the registers of 2^tpr_log2 threads, each
+// holding up to CPT 16-byte chunks (chunk c of the row sits in thread c % tpr,
+// slot c / tpr, so every load instruction of a warp is fully coalesced).
+// STATS = true writes the n_seg partials instead of normalising.
+// Register cap: 1024 / BLOCK blocks per SM, i.e. 64 registers per thread, so
+// an SM keeps at least 1024 threads x CPT x 16 B of loads in flight.
+template <typename TA, typename TW, int CPT, int BLOCK, bool STATS>
+__global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) rownorm_vec_kernel(const RowArgs a) {
+    constexpr int E = Chunk<TA>::E;
+    __shared__ float red[kMaxWarps][kFastMaxSeg];
+
+    int64_t b = blockIdx.x;
+    const int which = (b >= a.job[0].nblocks) ? 1 : 0;
+    if (which) b -= a.job[0].nblocks;
+    const RowJob J = pick_job(a, which);
+    const int tpr_log2 = J.tpr_log2;
+    const int tpr = 1 << tpr_log2;
+    const int lrow = threadIdx.x >> tpr_log2;
+    const int t = threadIdx.x & (tpr - 1);
+    const int64_t row = b * J.rows_per_cta + lrow;
+    const bool active = row < J.rows;
+    const int nchunks = J.nchunks;
+
+    // 1. issue every load of the row before any arithmetic
+    const uint8_t *xr = J.x + (active ? row : 0) * J.ld_bytes;
+    uint4 v[CPT];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * tpr + t;
+        if (active && c < nchunks) v[i] = ld_stream(xr + (int64_t)c * 16);
+        else v[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    // 2. per-thread partial sum of squares of each segment
+    float acc[kFastMaxSeg];
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) acc[j] = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * tpr + t;
+        float f[E];
+        Chunk<TA>::unpack(v[i], f);
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+        // floor(c / seg_chunks): (c + 0.5) / seg_chunks is never an integer, and
+        // the fp32 error stays below 0.5 / seg_chunks for c < 2^22 (host-checked)
+        const int seg = __float2int_rz(((float)c + 0.5f) * J.inv_seg_chunks);
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j) acc[j] += (j == seg) ? s : 0.f;
+    }
+
+    // 3. reduce each segment over the threads of the row (fixed tree)
+    const int n_seg = a.n_seg;
+    const int lanes = tpr < 32 ? tpr : 32;
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) {
+        if (j < n_seg) {
+            for (int off = lanes >> 1; off > 0; off >>= 1)
+                acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        }
+    }
+    if (tpr > 32) {  // uniform per block: a block serves one job
+        const int warp = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+            for (int j = 0; j < kFastMaxSeg; ++j)
+                if (j < n_seg) red[warp][j] = acc[j];
+        }
+        __syncthreads();
+        const int wpr = tpr >> 5;
+        const int w0 = lrow * wpr;
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j) {
+            if (j < n_seg) {
+                float s = 0.f;
+                for (int w = 0; w < wpr; ++w) s += red[w0 + w][j];
+                acc[j] = s;
+            }
+        }
+    }
+
+    if constexpr (STATS) {
+        if (active && t == 0) {
+            float *p = a.partial + row * n_seg;
+#pragma unroll
+            for (int j = 0; j < kFastMaxSeg; ++j)
+                if (j < n_seg) p[j] = acc[j];
+        }
+        return;
+    } else {
+        // 4. combine the segment statistics left to right, then scale
+        float S = 0.f;
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j)
+            if (j < n_seg) S += acc[j];
+        const float inv = rsqrtf(S / (float)J.d + a.eps);
+
+        // 5. apply the weights and store, one rounding per element
+        uint8_t *yr = J.y + (active ? row : 0) * J.ldo_bytes;
+        const TW *w = static_cast<const TW *>(J.w);
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = i * tpr + t;
+            if (active && c < nchunks) {
+                float f[E], wf[E];
+                Chunk<TA>::unpack_again(v[i], f);
+                load_weights<TW, E>(w + (int64_t)c * E, wf);
+#pragma unroll
+                for (int e = 0; e < E; ++e) f[e] = (f[e] * inv) * wf[e];
+                st_stream(yr + (int64_t)c * 16, Chunk<TA>::pack(f));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Element-wise kernel for any alignment, width and n_seg <= QKN_MAX_SEG: one
+// row per 256-thread block; each segment is reduced over the block in turn.
+// The row is read a second time (from L2) for the apply step.
+constexpr int kScalarBlock = 256;
+
+template <typename TA, typename TW, bool STATS>
+__global__ void __launch_bounds__(kScalarBlock) rownorm_scalar_kernel(const RowArgs a) {
+    __shared__ float warp_part[kScalarBlock / 32];
+    __shared__ float seg_total[QKN_MAX_SEG];
+
+    int64_t b = blockIdx.x;
+    const int which = (b >= a.job[0].rows) ? 1 : 0;
+    if (which) b -= a.job[0].rows;
+    const RowJob J = pick_job(a, which);
+    const TA *x = reinterpret_cast<const TA *>(J.x + b * J.ld_bytes);
+    const int d = J.d, n_seg = a.n_seg, seg_len = d / n_seg;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    for (int j = 0; j < n_seg; ++j) {
+        float s = 0.f;
+        for (int i = threadIdx.x; i < seg_len; i += kScalarBlock) {
+            const float f = to_f32<TA>(x[j * seg_len + i]);
+            s = fmaf(f, f, s);
+        }
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) warp_part[warp] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float tot = 0.f;
+            for (int w2 = 0; w2 < kScalarBlock / 32; ++w2) tot += warp_part[w2];
+            seg_total[j] = tot;
+        }
+        __syncthreads();
+    }
+
+    if constexpr (STATS) {
+        for (int j = threadIdx.x; j < n_seg; j += kScalarBlock) a.partial[b * n_seg + j] = seg_total[j];
+    } else {
+        float S = 0.f;
+        for (int j = 0; j < n_seg; ++j) S += seg_total[j];
+        const float inv = rsqrtf(S / (float)d + a.eps);
+        TA *y = reinterpret_cast<TA *>(J.y + b * J.ldo_bytes);
+        const TW *w = static_cast<const TW *>(J.w);
+        for (int i = threadIdx.x; i < d; i += kScalarBlock)
+            y[i] = from_f32<TA>((to_f32<TA>(x[i]) * inv) * to_f32<TW>(w[i]));
+    }
+}
+
+}  // namespace qkn

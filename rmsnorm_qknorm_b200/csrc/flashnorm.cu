@@ -1034,7 +1034,7 @@ extern "C" QKN_API qkn_status flashnorm_proj_noalloc(const void *x, const void *
     if (qkn_status st = noalloc_scratch(&inv)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (qkn_status st = launch_inv_rms(x, inv, M, K, eps, s)) return st;
-    return launch_gemm(x, W_folded, y, inv, M, N, K, eps, nullptr, s);
+    return launch_gemm(x, W_folded, y, inv, M, N, K, eps, nullptr, s, false, /*after_stats=*/true);
 }
 
 // ===================================================== RMSNorm elimination

@@ -151,7 +151,7 @@ thread_local uint64_t t_fault_wait_ns = 0;
 // One instantiation of the staged kernel, launched with programmatic stream
 // serialisation, so back-to-back launches overlap one grid's launch and
 // setup with the previous one's tail.
-template <typename TA, typename TW, bool STATS, bool NARROW>
+template <typename TA, typename TW, bool STATS, int FLAVOR>
 qkn_status launch_staged_kernel(const staged::Args &a, int grid, int smem, cudaStream_t s) {
     // the attribute is a cap: set once per device to the whole budget the
     // geometry ever asks for
@@ -160,7 +160,7 @@ qkn_status launch_staged_kernel(const staged::Args &a, int grid, int smem, cudaS
     cudaGetDevice(&dev);
     const bool known = dev >= 0 && dev < 64;
     if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(staged::rownorm_staged_kernel<TA, TW, STATS, NARROW>,
+        cudaError_t e = cudaFuncSetAttribute(staged::rownorm_staged_kernel<TA, TW, STATS, FLAVOR>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, QKN_STAGED_SMEM_LIMIT);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rownorm_staged_kernel)");
         if (known) attr_set[dev].store(true, std::memory_order_release);
@@ -176,7 +176,7 @@ qkn_status launch_staged_kernel(const staged::Args &a, int grid, int smem, cudaS
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, staged::rownorm_staged_kernel<TA, TW, STATS, NARROW>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, staged::rownorm_staged_kernel<TA, TW, STATS, FLAVOR>, a);
     if (e != cudaSuccess) return cuda_fail(e, "rownorm_staged_kernel launch");
     return check_launch("rownorm_staged_kernel launch");
 }
@@ -229,10 +229,18 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     }
     const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes);
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
-    bool narrow = false;
-    for (int i = 0; i < njobs; ++i) narrow = narrow || a.job[i].narrow_cpl != 0;
-    if (narrow) return launch_staged_kernel<TA, TW, STATS, true>(a, (int)grid, smem, s);
-    return launch_staged_kernel<TA, TW, STATS, false>(a, (int)grid, smem, s);
+    // the 512-chunk flavour (row kept in registers) is bit-identical to the
+    // generic one; it wins on long launches (131072 + 131072 rows: 729 -> 702
+    // us, 65536 + 65536: 1.5 %) and loses on short ones (32768 + 32768: +8 %),
+    // so it is used from 131072 rows per launch
+    bool narrow = false, all512 = rows * njobs >= 131072;
+    for (int i = 0; i < njobs; ++i) {
+        narrow = narrow || a.job[i].narrow_cpl != 0;
+        all512 = all512 && a.job[i].nchunks == 512;
+    }
+    if (narrow) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorNarrow>(a, (int)grid, smem, s);
+    if (all512) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorRow512>(a, (int)grid, smem, s);
+    return launch_staged_kernel<TA, TW, STATS, staged::kFlavorGeneric>(a, (int)grid, smem, s);
 }
 
 template <typename TA, typename TW, bool STATS>

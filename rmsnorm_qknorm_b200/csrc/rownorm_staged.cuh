@@ -183,53 +183,12 @@ __device__ __forceinline__ void apply_chunk(const uint4 &v, int c, float2 inv2, 
 // parked in the warp's [8][32] scratch `part` whenever a segment ends; the 8
 // slots are reduced over the warp by recursive halving (lanes 4j .. 4j+3 end
 // with segment j) and the segments added left to right.  Returns S.
-template <typename TA, bool STATS>
-__device__ __forceinline__ float row_statistic(const Args &a, const Job &J, const uint8_t *srow, int64_t row,
-                                               int lane, float *part) {
-    const int nchunks = J.nchunks;
+// Reduces the warp's parked segment sums (scratch [8][32]) by recursive
+// halving over the lanes (lanes 4j .. 4j+3 end with segment j), adds the
+// segments left to right and returns S; STATS stores the segment sums.
+template <bool STATS>
+__device__ __forceinline__ float finish_statistic(const Args &a, float *part, int64_t row, int lane) {
     const int n_seg = a.n_seg;
-    const int sc = J.seg_chunks;
-#pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
-    float2 cur = make_float2(0.f, 0.f);
-    int cur_seg = 0, next_bound = sc;
-    int c0 = 0;
-    constexpr int G = 32 * kUnroll;  // chunks per group
-    if (nchunks >= G) {
-        // groups of kUnroll chunks per lane; the next group's loads are issued
-        // before the current group's arithmetic
-        uint4 vn[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) vn[u] = *reinterpret_cast<const uint4 *>(srow + (u * 32 + lane) * 16);
-        for (; c0 + G <= nchunks; c0 += G) {
-            uint4 v[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) v[u] = vn[u];
-            if (c0 + 2 * G <= nchunks) {
-#pragma unroll
-                for (int u = 0; u < kUnroll; ++u)
-                    vn[u] = *reinterpret_cast<const uint4 *>(srow + (c0 + G + u * 32 + lane) * 16);
-            }
-            float2 sq[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) sq[u] = chunk_sumsq<TA>(v[u]);
-            if (c0 + (kUnroll - 1) * 32 + lane < next_bound) {  // the whole group is in the current segment
-#pragma unroll
-                for (int u = 0; u < kUnroll; ++u) cur = __fadd2_rn(cur, sq[u]);
-            } else {
-#pragma unroll
-                for (int u = 0; u < kUnroll; ++u)
-                    accumulate(sq[u], c0 + u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
-            }
-        }
-    }
-    for (; c0 < nchunks; c0 += 32) {
-        const int c = c0 + lane;
-        if (c < nchunks)
-            accumulate(chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)), c, cur, cur_seg,
-                       next_bound, sc, part, lane);
-    }
-    part[cur_seg * 32 + lane] = cur.x + cur.y;
     __syncwarp();
 
     float S = 0.f;
@@ -272,6 +231,55 @@ __device__ __forceinline__ float row_statistic(const Args &a, const Job &J, cons
     return S;
 }
 
+template <typename TA, bool STATS>
+__device__ __forceinline__ float row_statistic(const Args &a, const Job &J, const uint8_t *srow, int64_t row,
+                                               int lane, float *part) {
+    const int nchunks = J.nchunks;
+    const int sc = J.seg_chunks;
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
+    float2 cur = make_float2(0.f, 0.f);
+    int cur_seg = 0, next_bound = sc;
+    int c0 = 0;
+    constexpr int G = 32 * kUnroll;  // chunks per group
+    if (nchunks >= G) {
+        // groups of kUnroll chunks per lane; the next group's loads are issued
+        // before the current group's arithmetic
+        uint4 vn[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) vn[u] = *reinterpret_cast<const uint4 *>(srow + (u * 32 + lane) * 16);
+        for (; c0 + G <= nchunks; c0 += G) {
+            uint4 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) v[u] = vn[u];
+            if (c0 + 2 * G <= nchunks) {
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    vn[u] = *reinterpret_cast<const uint4 *>(srow + (c0 + G + u * 32 + lane) * 16);
+            }
+            float2 sq[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) sq[u] = chunk_sumsq<TA>(v[u]);
+            if (c0 + (kUnroll - 1) * 32 + lane < next_bound) {  // the whole group is in the current segment
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) cur = __fadd2_rn(cur, sq[u]);
+            } else {
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    accumulate(sq[u], c0 + u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
+            }
+        }
+    }
+    for (; c0 < nchunks; c0 += 32) {
+        const int c = c0 + lane;
+        if (c < nchunks)
+            accumulate(chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)), c, cur, cur_seg,
+                       next_bound, sc, part, lane);
+    }
+    part[cur_seg * 32 + lane] = cur.x + cur.y;
+    return finish_statistic<STATS>(a, part, row, lane);
+}
+
 // Statistic of a narrow row (32 * CPL chunks, CPL <= 4) whose segments are
 // whole groups of lanes: lane l sums its CPL contiguous chunks l*CPL ..
 // l*CPL + CPL - 1 (all in segment l / LPS, LPS = 32 / n_seg lanes per
@@ -303,16 +311,54 @@ __device__ __forceinline__ float narrow_statistic(const uint8_t *srow, int lane,
     return S;
 }
 
+// Kernel flavours, chosen per launch from the rows' shapes so that each
+// keeps only the register budget of the paths it can take.
+constexpr int kFlavorGeneric = 0;  // any row
+constexpr int kFlavorNarrow = 1;   // some rows take the narrow statistic
+constexpr int kFlavorRow512 = 2;   // every row is 512 chunks (4096 bf16 / 2048 fp32)
+
+// Rows of exactly 512 chunks: a lane's 16 chunks stay in registers from the
+// statistic to the apply, so the row is read from shared memory once.  The
+// arithmetic and its order are those of row_statistic and the apply below.
+template <typename TA, bool STATS>
+__device__ __forceinline__ float row512(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
+                                        int64_t row, int lane, float *part) {
+    constexpr int U = 16;
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = *reinterpret_cast<const uint4 *>(srow + (u * 32 + lane) * 16);
+    const int sc = J.seg_chunks;
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
+    float2 cur = make_float2(0.f, 0.f);
+    int cur_seg = 0, next_bound = sc;
+#pragma unroll
+    for (int u = 0; u < U; ++u) accumulate(chunk_sumsq<TA>(v[u]), u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
+    part[cur_seg * 32 + lane] = cur.x + cur.y;
+    const float S = finish_statistic<STATS>(a, part, row, lane);
+    if constexpr (!STATS) {
+        const float inv = rsqrtf(S / (float)J.d + a.eps);
+        const float2 inv2 = make_float2(inv, inv);
+        uint8_t *yr = J.y + row * J.ldo_bytes;
+#pragma unroll
+        for (int u = 0; u < U; ++u) apply_chunk<TA>(v[u], u * 32 + lane, inv2, wsm, 512, yr);
+    }
+    return S;
+}
+
 // One row held in shared memory, processed by one warp.  `part` is the warp's
-// [8][32] scratch for lane partials; `wsm` the job's fp32 weights.  NARROW:
-// the launch has narrow rows (the narrow statistic is compiled in; launches
-// without them keep the wide path alone, and its register budget).
-template <typename TA, bool STATS, bool NARROW>
+// [8][32] scratch for lane partials; `wsm` the job's fp32 weights.  FLAVOR
+// selects which statistic paths are compiled in (kFlavor*).
+template <typename TA, bool STATS, int FLAVOR>
 __device__ __forceinline__ void process_row(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
                                             int64_t row, int lane, float *part) {
     const int nchunks = J.nchunks;
+    if constexpr (FLAVOR == kFlavorRow512) {
+        row512<TA, STATS>(a, J, srow, wsm, row, lane, part);
+        return;
+    }
     float S;
-    if (NARROW && J.narrow_cpl != 0) {
+    if (FLAVOR == kFlavorNarrow && J.narrow_cpl != 0) {
         const int n_seg = a.n_seg;
         float seg;
         if (J.narrow_cpl == 1) S = narrow_statistic<TA, 1>(srow, lane, n_seg, seg);
@@ -372,7 +418,7 @@ __device__ __forceinline__ void issue_tile(const Args &a, int64_t tile, int64_t 
         bulk_g2s(dst + r * J.row_bytes, J.x + (row0 + r) * J.ld_bytes, (uint32_t)J.row_bytes, fb);
 }
 
-template <typename TA, typename TW, bool STATS, bool NARROW>
+template <typename TA, typename TW, bool STATS, int FLAVOR>
 __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int W = a.warps, SB = a.stage_bytes;
@@ -490,7 +536,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
         const uint8_t *sbase = smem + (size_t)stage * SB;
         const float4 *wsm = reinterpret_cast<const float4 *>(wbase + J.w_offset);
         for (int r = 0; r < nrows; ++r)
-            process_row<TA, STATS, NARROW>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
+            process_row<TA, STATS, FLAVOR>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
         __syncwarp();
         // refill this stage with the warp's tile k + spw
         const int64_t next = tile + spw * step;

@@ -262,3 +262,18 @@ def test_narrow_rows(cuda_lib, dtype, d, n_seg):
     assert torch.equal(y.view(torch.int16) if dtype == torch.bfloat16 else y,
                        y3.view(torch.int16) if dtype == torch.bfloat16 else y3)
     assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials d={d}")
+
+
+def test_long_launch_flavour_matches_short_launch(cuda_lib):
+    # 65536 + 65536 rows of 4096 bf16 run the register-resident flavour; the same rows
+    # in a short launch run the generic one: outputs must agree bit for bit
+    inp = W.make_qknorm_inputs("long_context", seed=5, device=DEV, tokens=65536)
+    qo, ko = run_pair(inp)
+    n = 777
+    qs, ks = qk.qknorm_fused(inp["q"][:n], inp["k"][:n], inp["wq"], inp["wk"], inp["eps"], inp["n_seg"])
+    torch.cuda.synchronize()
+    assert torch.equal(qo[:n].view(torch.int16), qs.view(torch.int16))
+    assert torch.equal(ko[:n].view(torch.int16), ks.view(torch.int16))
+    g = torch.Generator().manual_seed(1)
+    rows = torch.randint(0, 65536, (64,), generator=g).to(DEV)
+    check(qo[rows], inp["q"][rows], inp["wq"], inp["eps"], "long launch q sampled")

@@ -200,8 +200,10 @@ QKN_API qkn_status flashnorm_fold_weights(const void *w, const void *W, void *W_
  *   y[m][n] = inv[m] * sum_k x[m][k] * W'[n][k]   fp32 accumulate, bf16 out
  *
  * x          [M][K] bf16, row-major (K contiguous)
- * W_folded   [N][K] bf16 (K contiguous, out_k_major == 1 of the fold);
- *            w_k_major must be 1 (0 returns QKN_ERR_UNSUPPORTED)
+ * W_folded   w_k_major = 1: [N][K] bf16 (K contiguous, out_k_major == 1 of
+ *            the fold, the layout the tensor cores read); w_k_major = 0:
+ *            [K][N] bf16 (row-major, out_k_major == 0), copied K-major into a
+ *            stream-ordered temporary first (an extra pass over W')
  * y          [M][N] bf16, row-major
  * inv_rms    optional [M] fp32 precomputed 1/rms (then used as given)
  * inv_rms_out optional [M] fp32; when inv_rms is NULL and this is given, a
@@ -308,6 +310,8 @@ QKN_API qkn_status qkv_norm_proj(const void *x, const void *W_folded, void *y,
  *
  * Limits and caveats:
  * - M <= 262144 rows; larger M returns QKN_ERR_SHAPE before any launch.
+ * - W_folded must be K-major (w_k_major = 1): a row-major W' would need a
+ *   temporary copy, so w_k_major = 0 returns QKN_ERR_UNSUPPORTED.
  * - Every call on a GPU shares the one array: calls that overlap on the GPU
  *   (e.g. on two streams at once) race on it and must be serialised by the
  *   caller.  Each call writes the entries it reads, so the array's leftover

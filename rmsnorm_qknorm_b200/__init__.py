@@ -299,18 +299,22 @@ def flashnorm_fold_weights(w: torch.Tensor, W: torch.Tensor, *, k_major: bool = 
 
 def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *,
                    inv_rms: torch.Tensor | None = None, inv_rms_out: torch.Tensor | None = None,
-                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y [M, N] = (x [M, K] @ W_folded[N, K]^T) * 1/rms(x), bf16 in/out, fp32 accumulate."""
+                   out: torch.Tensor | None = None, k_major: bool = True, stream=None) -> torch.Tensor:
+    """y [M, N] = (x [M, K] @ W') * 1/rms(x), bf16 in/out, fp32 accumulate.
+
+    W_folded is [N, K] (``k_major=True``, the layout the tensor cores read) or
+    [K, N] (``k_major=False``: copied K-major inside the call first).
+    """
     _cuda(x, "x")
     _cuda(W_folded, "W_folded")
     if x.dim() != 2 or not x.is_contiguous() or x.dtype != torch.bfloat16:
         raise ValueError("x must be a contiguous bf16 [M, K] tensor")
     if W_folded.dim() != 2 or not W_folded.is_contiguous() or W_folded.dtype != torch.bfloat16:
-        raise ValueError("W_folded must be a contiguous bf16 [N, K] tensor")
+        raise ValueError("W_folded must be a contiguous bf16 2-D tensor")
     M, K = x.shape
-    N, K2 = W_folded.shape
+    N, K2 = W_folded.shape if k_major else (W_folded.shape[1], W_folded.shape[0])
     if K2 != K:
-        raise ValueError(f"W_folded is [{N}, {K2}] but x has K={K}")
+        raise ValueError(f"W_folded has K={K2} but x has K={K}")
     for name, t in (("inv_rms", inv_rms), ("inv_rms_out", inv_rms_out)):
         if t is not None:
             _vec(t, name, M)
@@ -321,7 +325,7 @@ def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *
     elif tuple(out.shape) != (M, N) or not out.is_contiguous() or out.dtype != torch.bfloat16:
         raise ValueError("out must be a contiguous bf16 [M, N] tensor")
     st = load_library().flashnorm_proj(
-        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, N, K, 1, float(eps),
+        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, N, K, 1 if k_major else 0, float(eps),
         inv_rms.data_ptr() if inv_rms is not None else None,
         inv_rms_out.data_ptr() if inv_rms_out is not None else None, _stream(stream))
     _check("flashnorm_proj", st)

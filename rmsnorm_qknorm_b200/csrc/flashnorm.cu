@@ -63,6 +63,24 @@ __global__ void __launch_bounds__(256) fold_transpose_kernel(const TW *__restric
     }
 }
 
+// W [K][N] -> W^T [N][K] through a 64x64 shared tile (the projection reads
+// its weights K-major).
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ W,
+                                                             __nv_bfloat16 *__restrict__ Wt, int64_t K, int64_t N) {
+    __shared__ __nv_bfloat16 tile[kFoldTile][kFoldTile + 2];
+    const int64_t k0 = (int64_t)blockIdx.y * kFoldTile, n0 = (int64_t)blockIdx.x * kFoldTile;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
+    for (int r = ty; r < kFoldTile; r += 4) {
+        const int64_t k = k0 + r, n = n0 + tx;
+        if (k < K && n < N) tile[r][tx] = W[k * N + n];
+    }
+    __syncthreads();
+    for (int r = ty; r < kFoldTile; r += 4) {
+        const int64_t n = n0 + r, k = k0 + tx;
+        if (n < N && k < K) Wt[n * K + k] = tile[tx][r];
+    }
+}
+
 // ======================================================= row statistics
 
 // inv[m] = 1/sqrt(sum_k x[m][k]^2 / K + eps), one warp per row, 16-byte loads
@@ -922,23 +940,47 @@ extern "C" QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded
     if (K % 8 != 0 || N % 8 != 0)
         return fail(QKN_ERR_SHAPE, "flashnorm_proj: K=%lld and N=%lld must be multiples of 8", (long long)K,
                     (long long)N);
-    if (!w_k_major) return fail(QKN_ERR_UNSUPPORTED, "flashnorm_proj: W_folded must be K-major ([N][K])");
     if (inv_rms == nullptr && (!(eps >= 0.f) || isinf(eps)))
         return fail(QKN_ERR_EPS, "flashnorm_proj: eps must be finite and >= 0");
     if (!aligned(x, 16) || !aligned(W_folded, 16) || !aligned(y, 16) || (inv_rms && !aligned(inv_rms, 4)) ||
         (inv_rms_out && !aligned(inv_rms_out, 4)))
         return fail(QKN_ERR_ALIGN, "flashnorm_proj: x, W_folded and y must be 16-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // W' given row-major ([K][N]): a stream-ordered K-major copy first, before
+    // the statistics pass, so the projection's early reads (it overlaps that
+    // pass) only see finished data
+    const void *Wk = W_folded;
+    void *tmp = nullptr;
+    if (!w_k_major) {
+        const int64_t gx = (N + kFoldTile - 1) / kFoldTile, gy = (K + kFoldTile - 1) / kFoldTile;
+        if (gx > 0x7fffffffLL || gy > 65535) return fail(QKN_ERR_SHAPE, "flashnorm_proj: W_folded too large to transpose");
+        cudaError_t e = cudaMallocAsync(&tmp, (size_t)(N * K * 2), s);
+        if (e != cudaSuccess) return cuda_fail(e, "flashnorm_proj: K-major copy of W_folded");
+        transpose_bf16_kernel<<<dim3((unsigned)gx, (unsigned)gy), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(W_folded), static_cast<__nv_bfloat16 *>(tmp), K, N);
+        if (qkn_status st = check_launch("transpose_bf16_kernel launch")) {
+            cudaFreeAsync(tmp, s);
+            return st;
+        }
+        Wk = tmp;
+    }
+    qkn_status st;
     if (inv_rms == nullptr && inv_rms_out != nullptr) {
         // the caller's buffer is the workspace of a separate row-statistics
         // pass, which leaves the matmul's shared-memory bandwidth to the MMA
-        if (qkn_status st = launch_inv_rms(x, inv_rms_out, M, K, eps, s)) return st;
+        st = launch_inv_rms(x, inv_rms_out, M, K, eps, s);
         // FlashNorm's "RMS and matmul in parallel": the projection starts while
         // the statistics pass runs and waits for it only in its epilogue
-        return launch_gemm(x, W_folded, y, inv_rms_out, M, N, K, eps, nullptr, s, false, true);
+        if (st == QKN_OK) st = launch_gemm(x, Wk, y, inv_rms_out, M, N, K, eps, nullptr, s, false, true);
+    } else {
+        // with no 1/rms at all the GEMM computes it beside the matmul (no workspace)
+        st = launch_gemm(x, Wk, y, inv_rms, M, N, K, eps, nullptr, s);
     }
-    // with no 1/rms at all the GEMM computes it beside the matmul (no workspace)
-    return launch_gemm(x, W_folded, y, inv_rms, M, N, K, eps, nullptr, s);
+    if (tmp != nullptr) {
+        const cudaError_t e = cudaFreeAsync(tmp, s);
+        if (e != cudaSuccess && st == QKN_OK) st = cuda_fail(e, "flashnorm_proj: releasing the K-major copy");
+    }
+    return st;
 }
 
 extern "C" QKN_API qkn_status qkn_check_device(void *stream) {

@@ -125,7 +125,11 @@ def test_proj_validation(lib):
     assert f(P, P, P, 0, 256, 64, 1, 1e-6, None, None, None) == SHAPE
     assert f(P, P, P, 128, 250, 64, 1, 1e-6, None, None, None) == SHAPE   # N % 8
     assert f(P, P, P, 128, 256, 60, 1, 1e-6, None, None, None) == SHAPE   # K % 8
-    assert f(P, P, P, 128, 256, 64, 0, 1e-6, None, None, None) == UNSUP   # N-major W'
+    assert f(P, P, P, 128, 256, 64, 0, -1.0, None, None, None) == EPS     # row-major W' is validated too
+    # the no-allocation form cannot make the K-major copy a row-major W' needs
+    g = lib.flashnorm_proj_noalloc
+    g.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_int, ctypes.c_float, ctypes.c_void_p]
+    assert g(P, P, P, 128, 256, 64, 0, 1e-6, None) == UNSUP
     assert f(P, P, P, 128, 256, 64, 1, -1.0, None, None, None) == EPS
     assert f(P + 8, P, P, 128, 256, 64, 1, 1e-6, None, None, None) == ALIGN  # TMA needs 16 B
     assert "16-byte" in lib.qkn_last_error().decode()

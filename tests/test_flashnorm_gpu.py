@@ -147,3 +147,20 @@ def test_device_error_word_clear(cuda_lib):
     # the projection kernel's bounded waits never gave up in this process
     lib = qk.load_library()
     assert lib.qkn_check_device(None) == 0, lib.qkn_last_error()
+
+
+@pytest.mark.parametrize("in_kernel_stats", [False, True])
+def test_row_major_folded_weights(cuda_lib, in_kernel_stats):
+    # W' handed over row-major ([K, N]) is copied K-major inside the call: the result is the
+    # K-major call's, bit for bit
+    M, K, N = 300, 520, 776
+    x, w, Wm, eps = _inputs(M, K, N, seed=21)
+    xd = x.to(DEV)
+    Wk = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV), k_major=True)
+    Wr = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV), k_major=False)
+    kw = {} if in_kernel_stats else {"inv_rms_out": torch.empty(M, dtype=torch.float32, device=DEV)}
+    a = qk.flashnorm_proj(xd, Wk, eps, **kw)
+    b = qk.flashnorm_proj(xd, Wr, eps, k_major=False, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert frobenius_rel(b, oracle.norm_then_project(x, w, Wm, eps)) <= PROJ_FROB_TOL

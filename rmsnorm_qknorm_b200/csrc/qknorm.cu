@@ -229,17 +229,9 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     }
     const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes);
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
-    // the 512-chunk flavour (row kept in registers) is bit-identical to the
-    // generic one; it wins on long launches (131072 + 131072 rows: 729 -> 702
-    // us, 65536 + 65536: 1.5 %) and loses on short ones (32768 + 32768: +8 %),
-    // so it is used from 131072 rows per launch
-    bool narrow = false, all512 = rows * njobs >= 131072;
-    for (int i = 0; i < njobs; ++i) {
-        narrow = narrow || a.job[i].narrow_cpl != 0;
-        all512 = all512 && a.job[i].nchunks == 512;
-    }
+    bool narrow = false;
+    for (int i = 0; i < njobs; ++i) narrow = narrow || a.job[i].narrow_cpl != 0;
     if (narrow) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorNarrow>(a, (int)grid, smem, s);
-    if (all512) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorRow512>(a, (int)grid, smem, s);
     return launch_staged_kernel<TA, TW, STATS, staged::kFlavorGeneric>(a, (int)grid, smem, s);
 }
 

@@ -315,36 +315,6 @@ __device__ __forceinline__ float narrow_statistic(const uint8_t *srow, int lane,
 // keeps only the register budget of the paths it can take.
 constexpr int kFlavorGeneric = 0;  // any row
 constexpr int kFlavorNarrow = 1;   // some rows take the narrow statistic
-constexpr int kFlavorRow512 = 2;   // every row is 512 chunks (4096 bf16 / 2048 fp32)
-
-// Rows of exactly 512 chunks: a lane's 16 chunks stay in registers from the
-// statistic to the apply, so the row is read from shared memory once.  The
-// arithmetic and its order are those of row_statistic and the apply below.
-template <typename TA, bool STATS>
-__device__ __forceinline__ float row512(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
-                                        int64_t row, int lane, float *part) {
-    constexpr int U = 16;
-    uint4 v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) v[u] = *reinterpret_cast<const uint4 *>(srow + (u * 32 + lane) * 16);
-    const int sc = J.seg_chunks;
-#pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
-    float2 cur = make_float2(0.f, 0.f);
-    int cur_seg = 0, next_bound = sc;
-#pragma unroll
-    for (int u = 0; u < U; ++u) accumulate(chunk_sumsq<TA>(v[u]), u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
-    part[cur_seg * 32 + lane] = cur.x + cur.y;
-    const float S = finish_statistic<STATS>(a, part, row, lane);
-    if constexpr (!STATS) {
-        const float inv = rsqrtf(S / (float)J.d + a.eps);
-        const float2 inv2 = make_float2(inv, inv);
-        uint8_t *yr = J.y + row * J.ldo_bytes;
-#pragma unroll
-        for (int u = 0; u < U; ++u) apply_chunk<TA>(v[u], u * 32 + lane, inv2, wsm, 512, yr);
-    }
-    return S;
-}
 
 // One row held in shared memory, processed by one warp.  `part` is the warp's
 // [8][32] scratch for lane partials; `wsm` the job's fp32 weights.  FLAVOR
@@ -353,10 +323,6 @@ template <typename TA, bool STATS, int FLAVOR>
 __device__ __forceinline__ void process_row(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
                                             int64_t row, int lane, float *part) {
     const int nchunks = J.nchunks;
-    if constexpr (FLAVOR == kFlavorRow512) {
-        row512<TA, STATS>(a, J, srow, wsm, row, lane, part);
-        return;
-    }
     float S;
     if (FLAVOR == kFlavorNarrow && J.narrow_cpl != 0) {
         const int n_seg = a.n_seg;

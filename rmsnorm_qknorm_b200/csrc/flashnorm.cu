@@ -394,316 +394,6 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
 
 }  // namespace gemm
 
-// ============================================ tcgen05 GEMM, CTA pair (ii)
-//
-// The same projection on a cluster of two CTAs (two SMs of a TPC) that
-// compute one 256 x 256 tile together with tcgen05.mma.cta_group::2: each CTA
-// keeps its own 128 rows of x and its own 128 rows of W' for a k-block in
-// shared memory (32 KiB per stage instead of 48), the even CTA issues the
-// M = 256 MMAs that read both CTAs' tiles, and each CTA's tensor memory holds
-// the fp32 accumulator of its own 128 rows.  Per SM that is a third less
-// shared-memory traffic per FLOP, and six stages fit.  Both CTAs' TMA loads
-// complete their bytes on the even CTA's stage barrier; the even CTA's
-// commits arrive (multicast) on the stage and accumulator barriers of both
-// CTAs; the epilogue warps of both CTAs release the even CTA's accumulator
-// barrier.  The x tiles of the pair are also the rows the CTAs scale, so the
-// epilogue is the same as the single-CTA kernel's, with a 1/rms supplied.
-namespace gemm2 {
-
-constexpr int BM = 128;                                  // rows per CTA (256 per pair)
-constexpr int BN = 256;                                  // columns per pair tile
-constexpr int BN_CTA = 128;                              // W' rows loaded by each CTA
-constexpr int BK = 64;
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK * 2;                     // 16 KiB
-constexpr int B_BYTES = BN_CTA * BK * 2;                 // 16 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 32 KiB per CTA
-constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;        // bytes landing on the even CTA's barrier
-constexpr int ACC_COLS = BN;
-constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int THREADS = 256;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-7 row statistics
-constexpr int BAR_BYTES = 256;
-constexpr int INV_BYTES = 2 * BM * 4;                     // 1/rms of this CTA's rows, both accumulators
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + INV_BYTES + 1024;
-constexpr int GROUP_M = 8;                               // pair row blocks (of 256) per raster group
-
-static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-
-// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 D, M = 256, N = 256.
-constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                ((uint32_t)(256 >> 4) << 24);
-
-struct Args {
-    const float *inv_rms;  // [M] given 1/rms (compute_inv == 0 and unit_scale == 0)
-    float *inv_out;        // [M] optional: receives the 1/rms computed in-kernel
-    __nv_bfloat16 *y;      // [M][N]
-    int M, N, K;
-    int pm_blocks, n_blocks, k_blocks, num_tiles;  // pm: 256-row blocks of the pair
-    int unit_scale;
-    int compute_inv;       // 1: each CTA computes its rows' 1/rms from its x tiles
-    float eps;
-};
-
-__device__ __forceinline__ void tile_coords(int tile, const Args &g, int &pm, int &n) {
-    const int group_tiles = GROUP_M * g.n_blocks;
-    const int group = tile / group_tiles;
-    const int first = group * GROUP_M;
-    const int rows_in_group = min(g.pm_blocks - first, GROUP_M);
-    const int in_group = tile - group * group_tiles;
-    pm = first + in_group % rows_in_group;
-    n = in_group / rows_in_group;
-}
-
-// 2-D tensor copy into this CTA's shared memory whose bytes complete on the
-// barrier at `bar_cluster` (the even CTA's), for a CTA-pair MMA.  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                                 uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster) : "memory");
-}
-
-__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kInstrDesc), "r"(accumulate));
-}
-
-// Arrives, once these MMAs have completed, on the barrier at this offset in
-// both CTAs of the pair.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-    const uint16_t mask = 0x3;
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                 ::"r"(bar), "h"(mask) : "memory");
-}
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                           const Args g) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *full = bars, *empty = bars + STAGES;
-    uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
-    uint64_t *stats_ready = bars + 2 * STAGES + 4;       // odd CTA: its x tile of a stage has landed
-    uint64_t *stats_full = bars + 3 * STAGES + 4;        // this CTA's 1/rms of an accumulator published
-    uint64_t *inv_free = bars + 3 * STAGES + 6;          // this CTA's epilogue is done with an inv buffer
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 8);
-    float *inv_buf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + BAR_BYTES);  // [2][BM]
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
-    const bool leader = rank == 0;
-    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);   // even CTA: its producer's arrive + both CTAs' bytes
-            // the even CTA's multicast commit, plus this CTA's statistics warps when they read x
-            mbar_init(smem_u32(&empty[s]), g.compute_inv ? 3 : 1);
-            mbar_init(smem_u32(&stats_ready[s]), 1);  // odd CTA: relayed by the even CTA's MMA warp
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(smem_u32(&acc_full[a]), 1);   // the even CTA's multicast commit
-            mbar_init(smem_u32(&acc_empty[a]), 8);  // even CTA: 4 epilogue warps of each CTA
-            mbar_init(smem_u32(&stats_full[a]), 2); // this CTA's two statistics warps
-            mbar_init(smem_u32(&inv_free[a]), 4);   // this CTA's four epilogue warps
-        }
-        mbar_init_fence();
-    }
-    if (warp == 1) {  // whole warp, in both CTAs: the pair's tensor memory
-        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-    }
-    gemm::tc_fence_before();
-    cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
-    gemm::tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
-    if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer (both CTAs)
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int tile = pair; ok && tile < g.num_tiles; tile += num_pairs) {
-            int pm, n;
-            tile_coords(tile, g, pm, n);
-            for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &g_device_error)) { ok = false; break; }
-                if (lane == 0) {
-                    const uint32_t fb_local = smem_u32(&full[stage]);
-                    const uint32_t fb = map_to_rank(fb_local, 0);
-                    if (leader) mbar_arrive_expect_tx(fb_local, PAIR_STAGE_BYTES);
-                    uint8_t *sa = smem + stage * STAGE_BYTES;
-                    tma_load_2d_pair(smem_u32(sa), &tmap_x, kb * BK, pm * 2 * BM + (int)rank * BM, fb);
-                    tma_load_2d_pair(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, n * BN + (int)rank * BN_CTA, fb);
-                }
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
-        }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer (even CTA)
-        if (leader) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int it = 0;
-            bool ok = true;
-            for (int tile = pair; ok && tile < g.num_tiles; tile += num_pairs, ++it) {
-                const int acc = it & 1;
-                const uint32_t acc_phase = (it >> 1) & 1;
-                if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, &g_device_error)) break;
-                gemm::tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-                for (int kb = 0; kb < g.k_blocks; ++kb) {
-                    if (!mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
-                    gemm::tc_fence_after();
-                    if (lane == 0) {
-                        // both CTAs' tiles of this stage have landed: tell the odd CTA's statistics warps
-                        if (g.compute_inv) mbar_arrive_cluster(map_to_rank(smem_u32(&stats_ready[stage]), 1));
-                        const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
-                        const uint32_t b0 = a0 + A_BYTES;
-#pragma unroll
-                        for (int k = 0; k < BK / gemm::UMMA_K; ++k)
-                            umma_pair(d_tmem, gemm::sw128_kmajor_desc(a0 + k * 32),
-                                      gemm::sw128_kmajor_desc(b0 + k * 32), (kb | k) != 0 ? 1u : 0u);
-                        umma_commit_pair(smem_u32(&empty[stage]));  // frees the stage in both CTAs
-                    }
-                    __syncwarp();
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                }
-                if (!ok) break;
-                if (lane == 0) umma_commit_pair(smem_u32(&acc_full[acc]));  // both CTAs' accumulators ready
-                __syncwarp();
-            }
-        }
-    } else if (warp < 6) {
-        // ---------------------------------------------------------------- epilogue (warps 2..5, both CTAs)
-        const int quarter = warp & 3;
-        int it = 0;
-        for (int tile = pair; tile < g.num_tiles; tile += num_pairs, ++it) {
-            int pm, n;
-            tile_coords(tile, g, pm, n);
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase, &g_device_error)) break;
-            gemm::tc_fence_after();
-            const int row = pm * 2 * BM + (int)rank * BM + quarter * 32 + lane;
-            const bool row_ok = row < g.M;
-            float r;
-            if (g.unit_scale) {
-                r = 1.f;
-            } else if (g.compute_inv) {
-                if (!mbar_wait(smem_u32(&stats_full[acc]), acc_phase, &g_device_error)) break;
-                r = inv_buf[acc * BM + quarter * 32 + lane];
-            } else {
-                r = row_ok ? __ldg(g.inv_rms + row) : 0.f;
-            }
-            __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
-            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                gemm::tmem_ld_32cols(tbase + c * 32, v);
-                const int col0 = n * BN + c * 32;
-                if (row_ok) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int col = col0 + j * 8;
-                        if (col < g.N) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * r, __uint_as_float(v[8 * j + 1]) * r);
-                            o.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * r, __uint_as_float(v[8 * j + 3]) * r);
-                            o.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * r, __uint_as_float(v[8 * j + 5]) * r);
-                            o.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * r, __uint_as_float(v[8 * j + 7]) * r);
-                            *reinterpret_cast<uint4 *>(yrow + col) = o;
-                        }
-                    }
-                }
-            }
-            gemm::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (g.compute_inv) mbar_arrive(smem_u32(&inv_free[acc]));
-                mbar_arrive_cluster(map_to_rank(smem_u32(&acc_empty[acc]), 0));
-            }
-        }
-    } else if (g.compute_inv) {
-        // ---------------------------------------------------------------- row statistics (warps 6, 7)
-        // Each CTA sums the squares of its own 128 x rows over K from the x
-        // tiles streaming through its shared memory (the 128-byte swizzle
-        // only permutes the 16-byte chunks inside a row).  Lane l of warp sw
-        // owns rows sw*64 + l and sw*64 + l + 32.  The even CTA waits on its
-        // stage barrier; the odd CTA on the relay its MMA warp sends.
-        const int sw = warp - 6;
-        int stage = 0;
-        uint32_t phase = 0;
-        int it = 0;
-        bool ok = true;
-        for (int tile = pair; ok && tile < g.num_tiles; tile += num_pairs, ++it) {
-            int pm, n;
-            tile_coords(tile, g, pm, n);
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
-            float2 ssq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            for (int kb = 0; kb < g.k_blocks; ++kb) {
-                const bool landed = leader ? mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)
-                                           : mbar_wait_cluster(smem_u32(&stats_ready[stage]), phase, &g_device_error);
-                if (!landed) { ok = false; break; }
-                const uint8_t *a_tile = smem + stage * STAGE_BYTES;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int rr = sw * 64 + lane + 32 * i;
-                    const uint8_t *arow = a_tile + rr * (BK * 2);
-                    uint4 v[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4 *>(arow + ((j ^ (rr & 7)) * 16));
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float2 p0 = make_float2(bf16lo(v[j].x), bf16hi(v[j].x));
-                        const float2 p1 = make_float2(bf16lo(v[j].y), bf16hi(v[j].y));
-                        const float2 p2 = make_float2(bf16lo(v[j].z), bf16hi(v[j].z));
-                        const float2 p3 = make_float2(bf16lo(v[j].w), bf16hi(v[j].w));
-                        ssq[i] = __ffma2_rn(p0, p0, ssq[i]);
-                        ssq[i] = __ffma2_rn(p1, p1, ssq[i]);
-                        ssq[i] = __ffma2_rn(p2, p2, ssq[i]);
-                        ssq[i] = __ffma2_rn(p3, p3, ssq[i]);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&empty[stage]));
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            }
-            if (!ok) break;
-            // the inv buffer of this accumulator is free once this CTA's epilogue finished tile it - 2
-            if (!mbar_wait(smem_u32(&inv_free[acc]), acc_phase ^ 1u, &g_device_error)) break;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int rr = sw * 64 + lane + 32 * i;
-                const float inv = rsqrtf((ssq[i].x + ssq[i].y) / (float)g.K + g.eps);
-                inv_buf[acc * BM + rr] = inv;
-                const int row = pm * 2 * BM + (int)rank * BM + rr;
-                if (g.inv_out != nullptr && n == 0 && row < g.M) g.inv_out[row] = inv;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&stats_full[acc]));
-        }
-    }
-
-    gemm::tc_fence_before();
-    __syncthreads();
-    cluster_sync();  // the even CTA's MMAs (which read this CTA's tiles) are done in both CTAs
-    if (warp == 1) {
-        gemm::tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                     : "memory");
-    }
-}
-
-}  // namespace gemm2
 
 // ----------------------------------------------------------- host helpers
 
@@ -767,84 +457,13 @@ qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float
 
 namespace {
 
-// The CTA-pair kernel measured slower than the single-CTA kernel in same-box
-// A/B runs, so it is not the default; QKN_GEMM_PAIR=1 selects it.
-#ifndef QKN_GEMM_PAIR
-#define QKN_GEMM_PAIR 0
-#endif
-
-// The CTA-pair projection: inv (1/rms per row) given, or unit_scale.
-qkn_status launch_gemm_pair(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N,
-                            int64_t K, bool unit_scale, float eps, float *inv_out, cudaStream_t s) {
-    CUtensorMap tx, tw;
-    if (qkn_status st = make_tmap(&tx, x, M, K, gemm2::BM)) return st;
-    if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm2::BN_CTA)) return st;
-    gemm2::Args g;
-    g.inv_rms = inv;
-    g.y = static_cast<__nv_bfloat16 *>(y);
-    g.M = (int)M;
-    g.N = (int)N;
-    g.K = (int)K;
-    g.pm_blocks = (int)((M + 2 * gemm2::BM - 1) / (2 * gemm2::BM));
-    g.n_blocks = (int)((N + gemm2::BN - 1) / gemm2::BN);
-    g.k_blocks = (int)((K + gemm2::BK - 1) / gemm2::BK);
-    g.num_tiles = g.pm_blocks * g.n_blocks;
-    g.unit_scale = unit_scale ? 1 : 0;
-    g.compute_inv = (inv == nullptr && !unit_scale) ? 1 : 0;
-    g.inv_out = g.compute_inv ? inv_out : nullptr;
-    g.eps = eps;
-    static std::atomic<bool> attr_set[64];  // per device: the attribute has been set
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const bool known = dev >= 0 && dev < 64;
-    if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(gemm2::flashnorm_gemm_pair_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, gemm2::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(flashnorm_gemm_pair_kernel)");
-        if (known) attr_set[dev].store(true, std::memory_order_release);
-    }
-    // a persistent grid must fit at once: as many pairs as the device can
-    // keep resident together (two-SM clusters need both SMs of a pair free)
-    static std::atomic<int> max_clusters[64];  // per device; 0 until measured
-    int pairs = known ? max_clusters[dev].load(std::memory_order_relaxed) : 0;
-    if (pairs == 0) {
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr;
-        attr.id = cudaLaunchAttributeClusterDimension;
-        attr.val.clusterDim.x = 2;
-        attr.val.clusterDim.y = 1;
-        attr.val.clusterDim.z = 1;
-        cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
-        cfg.blockDim = dim3(gemm2::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = gemm2::SMEM_BYTES;
-        cfg.attrs = &attr;
-        cfg.numAttrs = 1;
-        int n = 0;
-        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm2::flashnorm_gemm_pair_kernel, &cfg);
-        if (e != cudaSuccess || n <= 0) {
-            cudaGetLastError();
-            n = sm_count() / 2;
-        }
-        pairs = n;
-        if (known) max_clusters[dev].store(n, std::memory_order_relaxed);
-    }
-    const int grid = 2 * (g.num_tiles < pairs ? g.num_tiles : pairs);
-    gemm2::flashnorm_gemm_pair_kernel<<<grid, gemm2::THREADS, gemm2::SMEM_BYTES, s>>>(tx, tw, g);
-    return check_launch("flashnorm_gemm_pair_kernel launch");
-}
-
 // inv == nullptr (and not unit_scale): the single-CTA kernel computes every
 // row's 1/rms itself (eps) and, when inv_out is given, stores it there.
 // after_stats: the launch just before on `s` is this library's statistics
 // pass writing `inv` (and nothing the projection reads before its epilogue),
 // so the projection is launched as its programmatic dependent and overlaps it.
-// With QKN_GEMM_PAIR the CTA-pair kernel is tried first (never overlapped).
 qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv, int64_t M, int64_t N, int64_t K,
                        float eps, float *inv_out, cudaStream_t s, bool unit_scale = false, bool after_stats = false) {
-    if (QKN_GEMM_PAIR && sm_count() >= 2) {
-        const qkn_status st = launch_gemm_pair(x, Wf, y, inv, M, N, K, unit_scale, eps, inv_out, s);
-        if (st != QKN_ERR_CUDA) return st;  // a launch the device refused falls through
-    }
     CUtensorMap tx, tw;
     if (qkn_status st = make_tmap(&tx, x, M, K, gemm::BM)) return st;
     if (qkn_status st = make_tmap(&tw, Wf, N, K, gemm::BN)) return st;

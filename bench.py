@@ -54,13 +54,16 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=QK_DEFAULT,
                     choices=["tiny", "decode", "prefill_gqa", "long_context", "flashnorm_proj",
-                             "qkv_proj_qknorm"])
+                             "qkv_proj_qknorm", "tp_qknorm"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--strong", action="store_true",
                     help="split one batch over the ranks (strong scaling) instead of one batch per rank")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the QK-Norm workload's tokens per GPU (smaller cases for profiling)")
+    ap.add_argument("--tp-shards", type=int, default=None,
+                    help="tp_qknorm: on one GPU, time one rank's share of an S-way split "
+                         "(its kernels and local collectives; no interconnect transfer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline work budget")
     return ap.parse_args()
@@ -298,11 +301,12 @@ def run_reference(args):
         metric = "FlashNorm norm-then-project tokens/s (fp64 CPU oracle)"
         cfg = {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N}
     else:
-        wl = W.QKNORM_WORKLOADS[args.workload]
+        # the tensor-parallel layer computes the prefill GQA QK-Norm; the oracle computes it whole
+        wl = W.QKNORM_WORKLOADS["prefill_gqa" if args.workload == "tp_qknorm" else args.workload]
         inp = W.make_qknorm_inputs(wl, seed=0, tokens=min(wl.tokens, 8192))
         fn = lambda: cpu_baseline_qknorm(inp, 4.0)  # noqa: E731
         metric = "QK-Norm tokens/s (fp64 CPU oracle)"
-        cfg = {"workload": wl.name, "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk, "n_seg": wl.n_seg}
+        cfg = {"workload": args.workload, "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk, "n_seg": wl.n_seg}
     for _ in range(args.warmup):
         fn()
     vals = [fn() for _ in range(steps)]
@@ -706,6 +710,136 @@ def run_qkv(args, rank, world, local, pg):
         }), flush=True)
 
 
+def run_tp(args, rank, world, local, pg):
+    """Tensor-parallel QK-Norm of the prefill GQA layer (d split over the ranks):
+    SwiftQK's scalar exchange against the All-Gather form, per layer, on the device.
+    At one GPU a one-rank NCCL group runs the same collectives."""
+    import socket
+    import torch
+    import torch.distributed as dist
+    import rmsnorm_qknorm_b200 as qk
+    from rmsnorm_qknorm_b200 import tp
+    from rmsnorm_qknorm_b200 import workloads as W
+    qk.load_library()
+    own_group = False
+    if not dist.is_initialized():
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", local))
+        own_group = True
+    try:
+        _run_tp(args, rank, world, local, pg, torch, tp, W)
+    finally:
+        if own_group:
+            dist.destroy_process_group()
+
+
+def _run_tp(args, rank, world, local, pg, torch, tp, W):
+    import rmsnorm_qknorm_b200 as qk
+    wl = W.QKNORM_WORKLOADS["prefill_gqa"]
+    shards = args.tp_shards or world
+    if world > 1 and shards != world:
+        raise SystemExit("--tp-shards emulates a split on one GPU; with several ranks it must equal --gpus")
+    if shards < 1 or wl.dq % shards or wl.dk % shards:
+        raise SystemExit(f"dq={wl.dq} and dk={wl.dk} must split evenly over {shards} shards")
+    dq, dk = wl.dq // shards, wl.dk // shards
+    steps = args.steps if args.steps is not None else 200
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    inp = W.make_qknorm_inputs(wl, seed=0, device=dev)  # the same full rows on every rank
+    q = inp["q"][:, rank * dq:(rank + 1) * dq].contiguous()
+    k = inp["k"][:, rank * dk:(rank + 1) * dk].contiguous()
+    wq_s = inp["wq"][rank * dq:(rank + 1) * dq].contiguous()
+    wk_s = inp["wk"][rank * dk:(rank + 1) * dk].contiguous()
+    emulated = shards > world
+    if emulated:
+        # what one rank of the All-Gather form does once the slices have arrived:
+        # reassemble the rows from the gathered [shards, rows, d/shards] buffer,
+        # normalise them whole
+        T = wl.tokens
+        gq = inp["q"].view(T, shards, dq).permute(1, 0, 2).contiguous()
+        gk = inp["k"].view(T, shards, dk).permute(1, 0, 2).contiguous()
+
+        def allgather_local(_i):
+            qf = gq.permute(1, 0, 2).reshape(T, wl.dq)
+            kf = gk.permute(1, 0, 2).reshape(T, wl.dk)
+            qo, ko = qk.qknorm_fused(qf, kf, inp["wq"], inp["wk"], wl.eps, 1)
+            return qo[:, :dq], ko[:, :dk]
+    del inp["q"], inp["k"]
+    flows = {
+        # per-row scalar partials exchanged; q's exchange overlaps k's statistic
+        "swiftqk_overlap": lambda _i: tp.tp_qknorm(q, k, wq_s, wk_s, wl.dq, wl.dk, wl.eps, overlap=True),
+        # the same partials in one all-gather of [2, rows] per rank
+        "swiftqk_one_exchange": lambda _i: tp.tp_qknorm(q, k, wq_s, wk_s, wl.dq, wl.dk, wl.eps,
+                                                        overlap=False),
+        # all-gather of the activation slices, QK-Norm of the full rows
+        "allgather": allgather_local if emulated else
+        (lambda _i: tp.allgather_qknorm(q, k, inp["wq"], inp["wk"], wl.eps)),
+    }
+    warm = max(args.warmup, 3)
+    for i in range(warm):
+        for fn in flows.values():
+            fn(i)
+    barrier(pg)
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+        clocks.mark(True)
+    rounds = 5
+    per = max(steps // rounds, 1)
+    tot = dict.fromkeys(flows, 0.0)
+    for _ in range(rounds):  # interleaved, so that clock drift touches every flow alike
+        for name, fn in flows.items():
+            tot[name] += time_launches(fn, per, stream)[0]
+    steps = per * rounds
+    if clocks:
+        clocks.mark(False)
+    barrier(pg)
+    us = {name: max_over_ranks(t, pg) / steps * 1e3 for name, t in tot.items()}
+    clk = clocks.stop(gpu_index=local) if clocks else None
+    ms = us["swiftqk_overlap"] * 1e-3
+    pk, pk_kind = peaks()
+    local_bytes = wl.tokens * (dq + dk) * 2 * 2  # the shard's slices read and written once
+    achieved = local_bytes / (ms * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = W.make_qknorm_inputs(wl, seed=0, device="cpu", tokens=8192)
+        cpu = cpu_baseline_qknorm(host, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "Tensor-parallel QK-Norm tokens/s (SwiftQK scalar exchange) and latency reduction vs "
+                      "All-Gather QK-Norm",
+            "value": wl.tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "tp_qknorm", "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk,
+                       "parallelism": f"tp{shards} (q and k rows split over the ranks; NCCL group of {world})"
+                                      + (f"; one rank's share of a {shards}-way split emulated on one GPU: "
+                                         "kernels and local collectives only, no interconnect transfer"
+                                         if emulated else ""),
+                       "l2": "inputs larger than L2" if local_bytes > L2_BYTES else
+                             "per-rank slices fit in L2 (no flush)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "kernel": "whole tensor-parallel layer: two statistic launches, the exchange, "
+                                   "two apply launches",
+                         "algorithmic_bytes_per_launch": local_bytes,
+                         "note": "the statistic pass reads each slice a second time (3/2 of the algorithmic "
+                                 "bytes move)",
+                         "peak_source": f"{pk_kind} HBM copy bandwidth"},
+            "comparison": {"us_per_layer": us, "shards": shards, "emulated_share": emulated,
+                           "latency_reduction_vs_allgather": 1.0 - us["swiftqk_overlap"] / us["allgather"],
+                           "allgather": "all-gather of the q and k slices, rows reassembled, qknorm_fused "
+                                        "on the full rows"},
+            "cpu_baseline": cpu, "e2e": None, "clocks": clk,
+            # per step of each flow: two statistic and two apply launches (x2), one qknorm_fused
+            "gpu_launches": 9 * steps,
+        }), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -716,6 +850,8 @@ def main():
             run_flashnorm(args, rank, world, local, pg)
         elif args.workload == "qkv_proj_qknorm":
             run_qkv(args, rank, world, local, pg)
+        elif args.workload == "tp_qknorm":
+            run_tp(args, rank, world, local, pg)
         else:
             run_qknorm(args, rank, world, local, pg)
     finally:

@@ -12,7 +12,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("workload", ["tiny", "qkv_proj_qknorm"])
+@pytest.mark.parametrize("workload", ["tiny", "qkv_proj_qknorm", "tp_qknorm"])
 def test_reference_arm_json_line(workload):
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload,
                         "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True, text=True, timeout=300)

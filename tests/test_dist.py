@@ -120,3 +120,70 @@ def test_gather_without_process_group_is_local():
     from rmsnorm_qknorm_b200.tp import gather_partials
     g = gather_partials(torch.ones(3))
     assert tuple(g.shape) == (1, 3)
+
+
+def _slices_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from rmsnorm_qknorm_b200.tp import gather_slices
+        full = torch.arange(5 * 12, dtype=torch.float32).view(5, 12)
+        mine = full[:, rank * 6:(rank + 1) * 6].contiguous()
+        out[rank] = bool(torch.equal(gather_slices(mine), full))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gather_slices_reassembles_rows():
+    # the All-Gather baseline's exchange: every rank rebuilds the full rows in rank order
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(_slices_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    assert out[0] and out[1]
+
+
+def _tp_flow_worker(rank, world, port, overlap, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from rmsnorm_qknorm_b200 import tp
+        seen = []
+
+        def stats(x, o):  # stand-in for the statistic kernel: fp32 sum of squares of the slice
+            o.copy_((x.double() ** 2).sum(1).float())
+
+        def apply(x, w, parts_t, d_full, eps, inplace):  # stand-in for the apply kernel
+            seen.append(parts_t.clone())
+            return x * torch.rsqrt(parts_t.sum(1) / d_full + eps)[:, None] * w
+
+        tp._stats, tp._apply = stats, apply
+        g = torch.Generator().manual_seed(7)
+        q, k = torch.randn(6, 16, generator=g), torch.randn(6, 8, generator=g)
+        dq, dk = 16 // world, 8 // world
+        qs, ks = q[:, rank * dq:(rank + 1) * dq], k[:, rank * dk:(rank + 1) * dk]
+        wq, wk = torch.ones(dq), torch.ones(dk)
+        qo, ko = tp.tp_qknorm(qs, ks, wq, wk, 16, 8, 1e-6, overlap=overlap)
+        expect_q = torch.stack([(q[:, j * dq:(j + 1) * dq].double() ** 2).sum(1).float() for j in range(world)], 1)
+        expect_k = torch.stack([(k[:, j * dk:(j + 1) * dk].double() ** 2).sum(1).float() for j in range(world)], 1)
+        ref_q = qs * torch.rsqrt((q * q).mean(1) + 1e-6)[:, None]
+        ref_k = ks * torch.rsqrt((k * k).mean(1) + 1e-6)[:, None]
+        out[rank] = {
+            "parts_rank_order": bool(torch.equal(seen[0], expect_q) and torch.equal(seen[1], expect_k)),
+            "q_close": float((qo - ref_q).abs().max()), "k_close": float((ko - ref_k).abs().max()),
+        }
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+def test_tp_qknorm_exchange_flow(overlap):
+    # both exchange schedules of tp_qknorm (q's all-gather in flight while k's
+    # statistic runs, or one [2, rows] all-gather) hand every rank the partials
+    # of all ranks in rank order, and each rank's slice comes out normalised by
+    # the whole row's statistic
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(_tp_flow_worker, args=(world, _free_port(), overlap, out), nprocs=world, join=True)
+    for r in range(world):
+        assert out[r]["parts_rank_order"], r
+        assert out[r]["q_close"] < 1e-5 and out[r]["k_close"] < 1e-5, out[r]

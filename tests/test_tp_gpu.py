@@ -6,7 +6,8 @@
 * SwiftQK's tensor-parallel form emulated on one GPU: the row split into
   shard views, one partial per shard, the [shards, rows] partials combined in
   shard order -- within 1 bf16 ulp of the fp64 oracle.
-* tp_qknorm through torch.distributed with one NCCL rank.
+* tp_qknorm through torch.distributed with one NCCL rank, both exchange
+  schedules, and the All-Gather form it is compared with.
 * qkv_norm_proj (pre-attention RMSNorm eliminated) against the full oracle
   path RMSNorm(x) W followed by the q / k / v norms: relative Frobenius 1e-2.
 """
@@ -73,7 +74,7 @@ def _free_port() -> int:
 
 def test_tp_qknorm_single_rank_nccl(cuda_lib):
     import torch.distributed as dist
-    from rmsnorm_qknorm_b200.tp import tp_qknorm
+    from rmsnorm_qknorm_b200.tp import allgather_qknorm, tp_qknorm
     if dist.is_initialized():
         pytest.skip("a process group is already initialised")
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
@@ -81,9 +82,17 @@ def test_tp_qknorm_single_rank_nccl(cuda_lib):
     try:
         inp = W.make_qknorm_inputs("decode", seed=3, device=DEV, tokens=40)
         qo, ko = tp_qknorm(inp["q"], inp["k"], inp["wq"], inp["wk"], 5120, 5120, inp["eps"])
+        q1, k1 = tp_qknorm(inp["q"], inp["k"], inp["wq"], inp["wk"], 5120, 5120, inp["eps"], overlap=False)
+        # the All-Gather form the pages compare against: the same rows, normalised whole
+        qa, ka = allgather_qknorm(inp["q"], inp["k"], inp["wq"], inp["wk"], inp["eps"])
         torch.cuda.synchronize()
         assert_bf16_close(qo, oracle.rmsnorm(inp["q"].cpu(), inp["wq"].cpu(), inp["eps"]), "tp q")
         assert_bf16_close(ko, oracle.rmsnorm(inp["k"].cpu(), inp["wk"].cpu(), inp["eps"]), "tp k")
+        assert_bf16_close(qa, oracle.rmsnorm(inp["q"].cpu(), inp["wq"].cpu(), inp["eps"]), "all-gather q")
+        assert_bf16_close(ka, oracle.rmsnorm(inp["k"].cpu(), inp["wk"].cpu(), inp["eps"]), "all-gather k")
+        # the two exchange schedules combine the same partials in the same order
+        assert torch.equal(q1.view(torch.int16), qo.view(torch.int16))
+        assert torch.equal(k1.view(torch.int16), ko.view(torch.int16))
     finally:
         dist.destroy_process_group()
 

@@ -739,70 +739,101 @@ def run_tp(args, rank, world, local, pg):
 
 def _run_tp(args, rank, world, local, pg, torch, tp, W):
     import rmsnorm_qknorm_b200 as qk
+    from rmsnorm_qknorm_b200 import dist as qdist
     wl = W.QKNORM_WORKLOADS["prefill_gqa"]
     shards = args.tp_shards or world
     if world > 1 and shards != world:
         raise SystemExit("--tp-shards emulates a split on one GPU; with several ranks it must equal --gpus")
     if shards < 1 or wl.dq % shards or wl.dk % shards:
         raise SystemExit(f"dq={wl.dq} and dk={wl.dk} must split evenly over {shards} shards")
-    dq, dk = wl.dq // shards, wl.dk // shards
+    T, dq, dk = wl.tokens, wl.dq // shards, wl.dk // shards
     steps = args.steps if args.steps is not None else 200
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    inp = W.make_qknorm_inputs(wl, seed=0, device=dev)  # the same full rows on every rank
-    q = inp["q"][:, rank * dq:(rank + 1) * dq].contiguous()
-    k = inp["k"][:, rank * dk:(rank + 1) * dk].contiguous()
-    wq_s = inp["wq"][rank * dq:(rank + 1) * dq].contiguous()
-    wk_s = inp["wk"][rank * dk:(rank + 1) * dk].contiguous()
     emulated = shards > world
-    if emulated:
-        # what one rank of the All-Gather form does once the slices have arrived:
-        # reassemble the rows from the gathered [shards, rows, d/shards] buffer,
-        # normalise them whole
-        T = wl.tokens
-        gq = inp["q"].view(T, shards, dq).permute(1, 0, 2).contiguous()
-        gk = inp["k"].view(T, shards, dk).permute(1, 0, 2).contiguous()
+    local_bytes = T * (dq + dk) * 2 * 2  # the shard's slices read and written once
+    # enough input sets that consecutive steps never find their slices in L2
+    nsets = 1 if T * (dq + dk) * 2 > 2 * L2_BYTES else int(math.ceil(3 * L2_BYTES / (T * (dq + dk) * 2)))
+    sets = []
+    for si in range(nsets):
+        inp = W.make_qknorm_inputs(wl, seed=qdist.rank_seed(si, 0), device=dev)  # same rows on every rank
+        st = {"q": inp["q"][:, rank * dq:(rank + 1) * dq].contiguous(),
+              "k": inp["k"][:, rank * dk:(rank + 1) * dk].contiguous()}
+        if emulated:
+            # the buffers one rank of the All-Gather form holds once the slices arrived
+            st["gq"] = inp["q"].view(T, shards, dq).permute(1, 0, 2).contiguous()
+            st["gk"] = inp["k"].view(T, shards, dk).permute(1, 0, 2).contiguous()
+        if emulated or world == 1:
+            st["qf"], st["kf"] = inp["q"], inp["k"]  # whole rows, for the norm-only lower bound
+        sets.append(st)
+        wq, wk = inp["wq"], inp["wk"]
+        del inp
+    wq_s, wk_s = wq[rank * dq:(rank + 1) * dq].contiguous(), wk[rank * dk:(rank + 1) * dk].contiguous()
 
-        def allgather_local(_i):
-            qf = gq.permute(1, 0, 2).reshape(T, wl.dq)
-            kf = gk.permute(1, 0, 2).reshape(T, wl.dk)
-            qo, ko = qk.qknorm_fused(qf, kf, inp["wq"], inp["wk"], wl.eps, 1)
-            return qo[:, :dq], ko[:, :dk]
-    del inp["q"], inp["k"]
+    def allgather_local(st):
+        # reassemble the rows from the gathered [shards, rows, d/shards] buffer, normalise them whole
+        qf = st["gq"].permute(1, 0, 2).reshape(T, wl.dq)
+        kf = st["gk"].permute(1, 0, 2).reshape(T, wl.dk)
+        qo, ko = qk.qknorm_fused(qf, kf, wq, wk, wl.eps, 1)
+        return qo[:, :dq], ko[:, :dk]
+
     flows = {
         # per-row scalar partials exchanged; q's exchange overlaps k's statistic
-        "swiftqk_overlap": lambda _i: tp.tp_qknorm(q, k, wq_s, wk_s, wl.dq, wl.dk, wl.eps, overlap=True),
+        "swiftqk_overlap": lambda st: tp.tp_qknorm(st["q"], st["k"], wq_s, wk_s, wl.dq, wl.dk, wl.eps,
+                                                   overlap=True),
         # the same partials in one all-gather of [2, rows] per rank
-        "swiftqk_one_exchange": lambda _i: tp.tp_qknorm(q, k, wq_s, wk_s, wl.dq, wl.dk, wl.eps,
+        "swiftqk_one_exchange": lambda st: tp.tp_qknorm(st["q"], st["k"], wq_s, wk_s, wl.dq, wl.dk, wl.eps,
                                                         overlap=False),
         # all-gather of the activation slices, QK-Norm of the full rows
         "allgather": allgather_local if emulated else
-        (lambda _i: tp.allgather_qknorm(q, k, inp["wq"], inp["wk"], wl.eps)),
+        (lambda st: tp.allgather_qknorm(st["q"], st["k"], wq, wk, wl.eps)),
     }
+    if emulated or world == 1:
+        # the All-Gather form's normalisation alone, with the whole rows already
+        # in place (no transfer, no reassembly): a lower bound for that form
+        flows["allgather_norm_only"] = lambda st: qk.qknorm_fused(st["qf"], st["kf"], wq, wk, wl.eps, 1)
     warm = max(args.warmup, 3)
     for i in range(warm):
         for fn in flows.values():
-            fn(i)
+            fn(sets[i % nsets])
+    torch.cuda.synchronize()
+    # Each flow's timed layers are captured in one CUDA graph (collectives
+    # included) and replayed: the device time per layer, as a serving stack
+    # that replays captured layers sees it.  The same layers called one by one
+    # from Python are timed too (host-bound at these sizes).
+    graphs = {}
+    for name, fn in flows.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                fn(sets[i % nsets])
+        graphs[name] = g
+    for g in graphs.values():
+        g.replay()
+    torch.cuda.synchronize()
     barrier(pg)
     clocks = ClockSampler() if rank == 0 else None
     if clocks:
         clocks.start()
         clocks.mark(True)
-    rounds = 5
-    per = max(steps // rounds, 1)
-    tot = dict.fromkeys(flows, 0.0)
+    rounds = 3
+    dev_ms = dict.fromkeys(flows, 0.0)
+    eager_ms = dict.fromkeys(flows, 0.0)
     for _ in range(rounds):  # interleaved, so that clock drift touches every flow alike
+        for name in flows:
+            dev_ms[name] += time_launches(lambda _i: graphs[name].replay(), 1, stream)[0]
         for name, fn in flows.items():
-            tot[name] += time_launches(fn, per, stream)[0]
-    steps = per * rounds
+            eager_ms[name] += time_launches(lambda i: fn(sets[i % nsets]), steps, stream)[0]
     if clocks:
         clocks.mark(False)
     barrier(pg)
-    us = {name: max_over_ranks(t, pg) / steps * 1e3 for name, t in tot.items()}
+    n = rounds * steps
+    us = {name: max_over_ranks(t, pg) / n * 1e3 for name, t in dev_ms.items()}
+    us_eager = {name: max_over_ranks(t, pg) / n * 1e3 for name, t in eager_ms.items()}
     clk = clocks.stop(gpu_index=local) if clocks else None
+    del graphs  # graphs holding collectives go before the process group
     ms = us["swiftqk_overlap"] * 1e-3
     pk, pk_kind = peaks()
-    local_bytes = wl.tokens * (dq + dk) * 2 * 2  # the shard's slices read and written once
     achieved = local_bytes / (ms * 1e-3) / 1e9
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -812,16 +843,15 @@ def _run_tp(args, rank, world, local, pg, torch, tp, W):
         print(json.dumps({
             "metric": "Tensor-parallel QK-Norm tokens/s (SwiftQK scalar exchange) and latency reduction vs "
                       "All-Gather QK-Norm",
-            "value": wl.tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": n,
             "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "tp_qknorm", "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk,
+            "config": {"workload": "tp_qknorm", "tokens": T, "dq": wl.dq, "dk": wl.dk,
                        "parallelism": f"tp{shards} (q and k rows split over the ranks; NCCL group of {world})"
                                       + (f"; one rank's share of a {shards}-way split emulated on one GPU: "
                                          "kernels and local collectives only, no interconnect transfer"
                                          if emulated else ""),
-                       "l2": "inputs larger than L2" if local_bytes > L2_BYTES else
-                             "per-rank slices fit in L2 (no flush)"},
+                       "l2": f"{nsets} input sets cycled (inputs larger than L2 between reuses)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": None,
                          "kernel": "whole tensor-parallel layer: two statistic launches, the exchange, "
@@ -830,13 +860,19 @@ def _run_tp(args, rank, world, local, pg, torch, tp, W):
                          "note": "the statistic pass reads each slice a second time (3/2 of the algorithmic "
                                  "bytes move)",
                          "peak_source": f"{pk_kind} HBM copy bandwidth"},
-            "comparison": {"us_per_layer": us, "shards": shards, "emulated_share": emulated,
+            "comparison": {"us_per_layer": us, "us_per_layer_called_from_python": us_eager,
+                           "shards": shards, "emulated_share": emulated,
                            "latency_reduction_vs_allgather": 1.0 - us["swiftqk_overlap"] / us["allgather"],
+                           "latency_reduction_vs_norm_only": (1.0 - us["swiftqk_overlap"] / us["allgather_norm_only"]
+                                                              if "allgather_norm_only" in us else None),
                            "allgather": "all-gather of the q and k slices, rows reassembled, qknorm_fused "
-                                        "on the full rows"},
+                                        "on the full rows",
+                           "timing": "each flow's layers in one CUDA graph (collectives included), CUDA events "
+                                     "around the replay; the Python-called figures include the host"},
             "cpu_baseline": cpu, "e2e": None, "clocks": clk,
-            # per step of each flow: two statistic and two apply launches (x2), one qknorm_fused
-            "gpu_launches": 9 * steps,
+            # per step: two statistic and two apply launches in each SwiftQK flow, one qknorm_fused
+            # in each All-Gather flow; timed from the graphs and from Python
+            "gpu_launches": (8 + len(flows) - 2) * n * 2,
         }), flush=True)
 
 

@@ -103,6 +103,11 @@ qkn_status launch_cluster(const Tensor2 *ts, int njobs, int64_t rows, int n_seg,
     return check_launch("rownorm_cluster_kernel launch");
 }
 
+// Widest row (bytes, over the launch's jobs) that the register kernel takes
+// although the staged kernel's ring would hold it.
+constexpr int64_t kRegisterMaxRowBytes = 3072;
+constexpr int64_t kRegisterMaxRowBytesStats = 4096;
+
 // Vector-kernel configurations, tried in order: the first whose CPT covers
 // the widest row with at most `max_tpr` threads per row is used.
 struct VecCfg { int cpt, block; };
@@ -267,10 +272,16 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
         if (cfg < 0) vec = false;
     }
 
-    if (vec) {
-        int64_t max_row_bytes = 0;
-        for (int i = 0; i < njobs; ++i)
-            if (ts[i].d * (int64_t)sizeof(TA) > max_row_bytes) max_row_bytes = ts[i].d * (int64_t)sizeof(TA);
+    int64_t max_row_bytes = 0;
+    for (int i = 0; i < njobs; ++i)
+        if (ts[i].d * (int64_t)sizeof(TA) > max_row_bytes) max_row_bytes = ts[i].d * (int64_t)sizeof(TA);
+    // Narrow rows go to the register kernel: a stage of the staged kernel
+    // holds one row of the launch's widest job, so rows of a few hundred bytes
+    // would move in copies too small to keep HBM busy, and each warp would
+    // walk its rows one by one.  The bounds are where the two kernels measured
+    // even on B200 (rows of 1536 bf16 normalised, 2048 bf16 statistics only).
+    // The choice depends on the row widths alone, never on the row count.
+    if (vec && max_row_bytes > (STATS ? kRegisterMaxRowBytesStats : kRegisterMaxRowBytes)) {
         int64_t w_bytes = 0;
         for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
         int warps = 0, spw = 0, sb = 0;

@@ -8,7 +8,9 @@
 // d of the row's d_full elements normalises its slice once the n_part scalar
 // partial sums of the row (one per shard or segment) have been gathered:
 //   S = ((p_0 + p_1) + ...) + p_{n_part-1},   y_i = (x_i * rsqrt(S / d_full + eps)) * w_i
-// One warp per row; 16-byte accesses when the row layout allows.
+// 16-byte accesses when the row layout allows, with 2^tpr_log2 threads per
+// row (narrow rows share a warp, so a short row does not leave lanes idle);
+// otherwise one warp per row, element by element.
 namespace qkn {
 namespace {
 
@@ -17,10 +19,11 @@ __global__ void __launch_bounds__(256) apply_partials_kernel(const uint8_t *__re
                                                              const TW *__restrict__ w, const float *__restrict__ part,
                                                              int64_t rows, int d, int64_t ld_bytes,
                                                              int64_t ldo_bytes, int n_part, int64_t p_row,
-                                                             int64_t p_part, float d_full, float eps) {
-    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;  // whole warp leaves together
+                                                             int64_t p_part, float d_full, float eps, int tpr_log2) {
+    const int tpr = 1 << tpr_log2;
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> tpr_log2) + (threadIdx.x >> tpr_log2);
+    const int t = threadIdx.x & (tpr - 1);
+    if (row >= rows) return;  // no collective operations below
     float S = 0.f;
     for (int j = 0; j < n_part; ++j) S += __ldg(part + row * p_row + j * p_part);
     const float inv = rsqrtf(S / d_full + eps);
@@ -29,16 +32,16 @@ __global__ void __launch_bounds__(256) apply_partials_kernel(const uint8_t *__re
     if constexpr (VEC) {
         constexpr int E = Chunk<TA>::E;
         const int nchunks = d / E;
-        for (int c0 = 0; c0 < nchunks; c0 += 32 * 4) {
+        for (int c0 = 0; c0 < nchunks; c0 += tpr * 4) {
             uint4 v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int c = c0 + u * 32 + lane;
+                const int c = c0 + u * tpr + t;
                 v[u] = c < nchunks ? ld_stream(xr + (int64_t)c * 16) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int c = c0 + u * 32 + lane;
+                const int c = c0 + u * tpr + t;
                 if (c < nchunks) {
                     float f[E], wf[E];
                     Chunk<TA>::unpack(v[u], f);
@@ -52,7 +55,7 @@ __global__ void __launch_bounds__(256) apply_partials_kernel(const uint8_t *__re
     } else {
         const TA *xe = reinterpret_cast<const TA *>(xr);
         TA *ye = reinterpret_cast<TA *>(yr);
-        for (int i = lane; i < d; i += 32) ye[i] = from_f32<TA>((to_f32<TA>(xe[i]) * inv) * to_f32<TW>(w[i]));
+        for (int i = t; i < d; i += tpr) ye[i] = from_f32<TA>((to_f32<TA>(xe[i]) * inv) * to_f32<TW>(w[i]));
     }
 }
 
@@ -65,17 +68,25 @@ qkn_status launch_apply(const void *x, const void *w, void *y, int64_t rows, int
     const uintptr_t walign = (E * sizeof(TW)) < 16 ? E * sizeof(TW) : 16;
     const bool vec = aligned(x, 16) && aligned(y, 16) && (ld * es) % 16 == 0 && (ldo * es) % 16 == 0 &&
                      d % E == 0 && aligned(w, walign);
-    const int64_t blocks = (rows + 7) / 8;
+    // threads per row: enough for four chunks each, at most a warp
+    int tpr_log2 = 5;
+    if (vec) {
+        const int64_t per4 = (d / E + 3) / 4;
+        tpr_log2 = 0;
+        while (tpr_log2 < 5 && (int64_t(1) << tpr_log2) < per4) ++tpr_log2;
+    }
+    const int64_t rows_per_block = 256 >> tpr_log2;
+    const int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
     if (blocks > 0x7fffffffLL) return fail(QKN_ERR_SHAPE, "rmsnorm_apply_partials: too many rows");
     const uint8_t *xb = static_cast<const uint8_t *>(x);
     uint8_t *yb = static_cast<uint8_t *>(y);
     const TW *wt = static_cast<const TW *>(w);
     if (vec)
         apply_partials_kernel<TA, TW, true><<<(unsigned)blocks, 256, 0, s>>>(
-            xb, yb, wt, part, rows, (int)d, ld * (int64_t)es, ldo * (int64_t)es, n_part, p_row, p_part, (float)d_full, eps);
+            xb, yb, wt, part, rows, (int)d, ld * (int64_t)es, ldo * (int64_t)es, n_part, p_row, p_part, (float)d_full, eps, tpr_log2);
     else
         apply_partials_kernel<TA, TW, false><<<(unsigned)blocks, 256, 0, s>>>(
-            xb, yb, wt, part, rows, (int)d, ld * (int64_t)es, ldo * (int64_t)es, n_part, p_row, p_part, (float)d_full, eps);
+            xb, yb, wt, part, rows, (int)d, ld * (int64_t)es, ldo * (int64_t)es, n_part, p_row, p_part, (float)d_full, eps, tpr_log2);
     return check_launch("apply_partials_kernel launch");
 }
 

@@ -66,6 +66,19 @@ def test_apply_partials_fp32_and_unaligned(cuda_lib):
     assert_f32_close(y, oracle.rmsnorm(x.cpu(), w.cpu(), 1e-5), what="fp32 element path")
 
 
+@pytest.mark.parametrize("d,n_seg", [(8, 1), (64, 2), (136, 1), (1032, 3), (200, 4)])
+def test_apply_partials_row_widths(cuda_lib, d, n_seg):
+    # narrow rows share a warp (1, 2, 4 ... threads per row), 200 bf16 is not whole
+    # chunks per segment; 1000 rows leave a ragged last block
+    g = torch.Generator().manual_seed(d)
+    x = (torch.randn(1000, d, generator=g) * 3).to(torch.bfloat16).to(DEV)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16).to(DEV)
+    p = qk.rmsnorm_partial_stats(x, n_seg)
+    y = qk.rmsnorm_apply_partials(x, w, p, d, 1e-6)
+    torch.cuda.synchronize()
+    assert_bf16_close(y, oracle.rmsnorm(x.cpu(), w.cpu(), 1e-6), f"apply d={d} n_seg={n_seg}")
+
+
 def _free_port() -> int:
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -93,6 +106,15 @@ def test_tp_qknorm_single_rank_nccl(cuda_lib):
         # the two exchange schedules combine the same partials in the same order
         assert torch.equal(q1.view(torch.int16), qo.view(torch.int16))
         assert torch.equal(k1.view(torch.int16), ko.view(torch.int16))
+        # captured in a CUDA graph (collectives included) and replayed: the same bits
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            qg, kg = tp_qknorm(inp["q"], inp["k"], inp["wq"], inp["wk"], 5120, 5120, inp["eps"])
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(qg.view(torch.int16), qo.view(torch.int16))
+        assert torch.equal(kg.view(torch.int16), ko.view(torch.int16))
+        del g
     finally:
         dist.destroy_process_group()
 

@@ -434,7 +434,7 @@ def run_qknorm(args, rank, world, local, pg):
         h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size()
         e2e = {"value": global_tokens / (e_ms / args.e2e_steps * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
-               "note": "qknorm_fused_host on pinned host q,k: 32 MiB chunks uploaded, normalised and downloaded "
+               "note": "qknorm_fused_host on pinned host q,k: chunks of ~sqrt(bytes x 1.5 MB) uploaded, normalised and downloaded "
                         "with the three overlapped; outputs in pinned host memory, per step"}
 
     cpu = None

@@ -201,7 +201,7 @@ def qknorm_fused(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
     return q_out_t, k_out_t
 
 
-HOST_WORKSPACE_BYTES = 3 * 32 * 1024 * 1024
+HOST_WORKSPACE_BYTES = 3 * 64 * 1024 * 1024  # room for chunks up to 64 MiB
 
 
 def qknorm_fused_host(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,

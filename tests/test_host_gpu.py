@@ -44,6 +44,19 @@ def test_host_matches_device_call(cuda_lib, pinned, ws_rows):
     assert_bf16_close(qo, oracle.rmsnorm(inp["q"], inp["wq"], wl.eps), what="q")
 
 
+def test_host_default_workspace_several_chunks(cuda_lib):
+    # 3000 rows of 12 KiB: the default workspace holds 64 MiB chunks, but the
+    # chunk is sized from the bytes moved (16 MiB here), so three chunks run
+    wl = W.QKNORM_WORKLOADS["prefill_gqa"]
+    inp = W.make_qknorm_inputs(wl, seed=11, device="cpu", tokens=3000)
+    q, k = inp["q"].pin_memory(), inp["k"].pin_memory()
+    qo, ko = qk.qknorm_fused_host(q, k, inp["wq"].to(DEV), inp["wk"].to(DEV), wl.eps, wl.n_seg)
+    torch.cuda.synchronize()
+    rq, rk = _device_ref(inp, wl)
+    assert torch.equal(qo.view(torch.int16), rq.view(torch.int16))
+    assert torch.equal(ko.view(torch.int16), rk.view(torch.int16))
+
+
 def test_host_in_place_fp32_q_only(cuda_lib):
     wl = W.QKNORM_WORKLOADS["tiny"]
     inp = W.make_qknorm_inputs(wl, seed=3, device="cpu", tokens=50)

@@ -85,12 +85,13 @@ typedef enum {
  *
  * Alignment: any element-aligned pointers and pitches are accepted.  When
  * every row start is 16-byte aligned and each segment is a whole number of
- * 16-byte chunks, a vectorised kernel runs: for n_seg <= 8 and rows one
- * CTA holds, rows held in registers when the widest of q and k is at most
- * 3072 bytes (4096 for rmsnorm_partial_stats), else staged through shared
- * memory; for more segments or wider rows, each row spread over the CTAs
- * of a thread-block cluster that exchange only their per-segment partial
- * sums (rows up to 8 x 16384 bf16 / 8 x 8192 fp32 elements).  Otherwise a slower element-wise kernel computes the same
+ * 16-byte chunks, a vectorised kernel runs: rows held in registers when
+ * n_seg <= 8 and the widest of q and k is at most 3072 bytes (4096 for
+ * rmsnorm_partial_stats); else rows staged through shared memory while the
+ * widest row fits the staging ring (about 40 KiB, any n_seg); wider rows
+ * spread over the CTAs of a thread-block cluster that exchange only their
+ * per-segment partial sums (rows up to 8 x 16384 bf16 / 8 x 8192 fp32
+ * elements).  Otherwise a slower element-wise kernel computes the same
  * result.  Which kernel runs depends on the sizes, alignment and n_seg, never
  * on T.  The staged kernel is launched as a programmatic dependent: it
  * touches no global memory before the previous kernel on `stream` finished.

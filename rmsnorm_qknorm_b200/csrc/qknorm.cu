@@ -132,11 +132,13 @@ qkn_status launch_vec(RowArgs &a, int njobs, cudaStream_t s) {
 // Ring geometry for the staged kernel: stage = the widest row (rounded up to
 // 16 bytes); as many consumer warps (at most kMaxWarps) as allow two stages
 // per warp next to the fp32 weights within the shared-memory limit.  Returns
-// false when even 2 warps x 2 stages do not fit (the register kernel runs).
-bool staged_geometry(int64_t max_row_bytes, int64_t w_bytes, int *warps, int *spw, int *stage_bytes) {
+// false when even 2 warps x 2 stages do not fit (the register or cluster
+// kernel runs).  Each warp also keeps the segment scratch for n_seg.
+bool staged_geometry(int64_t max_row_bytes, int64_t w_bytes, int n_seg, int *warps, int *spw, int *stage_bytes) {
     const int64_t sb = (max_row_bytes + 15) / 16 * 16;
+    const int64_t scratch = (int64_t)staged::scratch_floats(n_seg) * 4;
     for (int w = staged::kMaxWarps; w >= 2; --w) {
-        const int64_t fixed = w_bytes + w * kFastMaxSeg * 32 * 4 + 8 * w * staged::kMaxStagesPerWarp;
+        const int64_t fixed = w_bytes + w * scratch + 8 * w * staged::kMaxStagesPerWarp;
         int64_t per_warp = (staged::kSmemLimit - fixed) / (w * sb);
         if (per_warp > staged::kMaxStagesPerWarp) per_warp = staged::kMaxStagesPerWarp;
         if (per_warp >= 2) {
@@ -202,6 +204,7 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     a.w_bytes = 0;
     a.wait_ns = kWaitTimeoutNs;
     a.fault_warp = -1;
+    a.scratch_floats = staged::scratch_floats(n_seg);
     if (t_fault_wait_ns != 0) {
         a.wait_ns = t_fault_wait_ns;
         a.fault_warp = 0;
@@ -225,15 +228,17 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
         J.rows_per_tile = stage_bytes / J.row_bytes;
         // narrow rows of 32, 64 or 128 chunks whose segments are whole power-of-two lane groups
         J.narrow_cpl = 0;
-        if (J.nchunks % 32 == 0 && J.nchunks <= 128) {
+        if (n_seg <= kFastMaxSeg && J.nchunks % 32 == 0 && J.nchunks <= 128) {
             const int cpl = J.nchunks / 32, lps = 32 / n_seg;
             if (lps * n_seg == 32 && (lps & (lps - 1)) == 0 && J.seg_chunks == cpl * lps) J.narrow_cpl = cpl;
         }
         J.ntiles = (rows + J.rows_per_tile - 1) / J.rows_per_tile;
         a.total_tiles += J.ntiles;
     }
-    const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes);
+    const int smem = staged::smem_bytes(a.warps, a.stages, a.stage_bytes, a.w_bytes, a.scratch_floats);
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
+    if (n_seg > kFastMaxSeg)
+        return launch_staged_kernel<TA, TW, STATS, staged::kFlavorManySeg>(a, (int)grid, smem, s);
     bool narrow = false;
     for (int i = 0; i < njobs; ++i) narrow = narrow || a.job[i].narrow_cpl != 0;
     if (narrow) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorNarrow>(a, (int)grid, smem, s);
@@ -281,11 +286,14 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
     // walk its rows one by one.  The bounds are where the two kernels measured
     // even on B200 (rows of 1536 bf16 normalised, 2048 bf16 statistics only).
     // The choice depends on the row widths alone, never on the row count.
-    if (vec && max_row_bytes > (STATS ? kRegisterMaxRowBytesStats : kRegisterMaxRowBytes)) {
+    // More than 8 segments (the register kernel stops at 8) take the staged
+    // kernel's many-segment statistic when its ring holds the rows.
+    const bool many = chunked && n_seg > kFastMaxSeg;
+    if ((vec && max_row_bytes > (STATS ? kRegisterMaxRowBytesStats : kRegisterMaxRowBytes)) || many) {
         int64_t w_bytes = 0;
         for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
         int warps = 0, spw = 0, sb = 0;
-        if (staged_geometry(max_row_bytes, w_bytes, &warps, &spw, &sb))
+        if (staged_geometry(max_row_bytes, w_bytes, n_seg, &warps, &spw, &sb))
             return launch_staged<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, warps, spw, sb, s);
     }
 

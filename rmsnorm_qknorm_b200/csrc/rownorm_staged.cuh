@@ -36,7 +36,10 @@ namespace qkn {
 // it crosses a segment boundary.  The eight slots are then reduced over the
 // warp by recursive halving (lane bit 4 splits segments 0-3 / 4-7, bit 3 and
 // bit 2 split further, bits 1 and 0 finish the sum), after which lanes
-// 4j .. 4j+3 hold segment j; the segments are combined left to right.
+// 4j .. 4j+3 hold segment j; the segments are combined left to right.  With
+// more than eight segments (up to 64) each segment has its own slot, lane j
+// adds slot j's 32 lane sums in lane order, and the segments are again
+// combined left to right.
 namespace staged {
 
 #ifndef QKN_STAGED_SMEM_LIMIT
@@ -84,11 +87,20 @@ struct Args {
     int w_bytes;      // fp32 weights of both jobs
     uint64_t wait_ns;  // limit of every mbarrier wait
     int fault_warp;   // testing only: this block*W+warp skips its first tile's copies (-1: none)
+    int scratch_floats;  // per warp: segment slots x their lane stride
 };
 
-// Shared memory: [ring][fp32 weights][full bars][W x 8 x 32 floats scratch]
-inline int smem_bytes(int warps, int stages, int stage_bytes, int w_bytes) {
-    return stages * stage_bytes + w_bytes + stages * 8 + warps * kFastMaxSeg * 32 * 4;
+// Segment slots of a warp's scratch: 8 x 32 floats for up to 8 segments; for
+// more, one slot per segment padded to 33 floats, so that lane j reading
+// slot j's 32 entries in turn touches a different bank from every other lane.
+constexpr int kManySegStride = 33;
+inline int scratch_floats(int n_seg) {
+    return n_seg <= kFastMaxSeg ? kFastMaxSeg * 32 : n_seg * kManySegStride;
+}
+
+// Shared memory: [ring][fp32 weights][full bars][W x scratch_floats scratch]
+inline int smem_bytes(int warps, int stages, int stage_bytes, int w_bytes, int scratch_per_warp) {
+    return stages * stage_bytes + w_bytes + stages * 8 + warps * scratch_per_warp * 4;
 }
 
 __device__ __forceinline__ Job pick(const Args &a, int which) {
@@ -152,10 +164,11 @@ __device__ __forceinline__ float2 chunk_sumsq(const uint4 &v) {
 
 // Adds a chunk's sum into the running pair sum, parking the running sum of
 // the segment being left whenever chunk c crosses a segment boundary.
+template <int STRIDE = 32>
 __device__ __forceinline__ void accumulate(float2 sq, int c, float2 &cur, int &cur_seg, int &next_bound,
                                            int seg_chunks, float *part, int lane) {
     while (c >= next_bound) {
-        part[cur_seg * 32 + lane] = cur.x + cur.y;
+        part[cur_seg * STRIDE + lane] = cur.x + cur.y;
         cur = make_float2(0.f, 0.f);
         ++cur_seg;
         next_bound += seg_chunks;
@@ -180,14 +193,10 @@ __device__ __forceinline__ void apply_chunk(const uint4 &v, int c, float2 inv2, 
     st_stream_batched(yr + (int64_t)c * 16, Pairs<TA>::put(p));
 }
 
-// Statistic of one row held in shared memory, by one warp (any width): lane
-// l adds its chunks l, l + 32, ... in order into a running pair sum that is
-// parked in the warp's [8][32] scratch `part` whenever a segment ends; the 8
-// slots are reduced over the warp by recursive halving (lanes 4j .. 4j+3 end
-// with segment j) and the segments added left to right.  Returns S.
-// Reduces the warp's parked segment sums (scratch [8][32]) by recursive
-// halving over the lanes (lanes 4j .. 4j+3 end with segment j), adds the
-// segments left to right and returns S; STATS stores the segment sums.
+// Up to 8 segments: reduces the warp's parked segment sums (scratch [8][32])
+// by recursive halving over the lanes (lanes 4j .. 4j+3 end with segment j),
+// adds the segments left to right and returns S; STATS stores the segment
+// sums.
 template <bool STATS>
 __device__ __forceinline__ float finish_statistic(const Args &a, float *part, int64_t row, int lane) {
     const int n_seg = a.n_seg;
@@ -233,13 +242,57 @@ __device__ __forceinline__ float finish_statistic(const Args &a, float *part, in
     return S;
 }
 
-template <typename TA, bool STATS>
+// More than 8 segments (up to 64): the lane sums were parked one slot per
+// segment (stride 33); lane j adds slot j's 32 entries in lane order (and
+// slot j + 32's), then the segments are added left to right.  Returns S;
+// STATS stores the segment sums.
+template <bool STATS>
+__device__ __forceinline__ float finish_many(const Args &a, const float *part, int64_t row, int lane) {
+    const int n_seg = a.n_seg;
+    __syncwarp();
+    float r0 = 0.f, r1 = 0.f;
+    if (lane < n_seg) {
+        const float *p = part + lane * kManySegStride;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) r0 += p[i];
+    }
+    if (lane + 32 < n_seg) {
+        const float *p = part + (lane + 32) * kManySegStride;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) r1 += p[i];
+    }
+    if constexpr (STATS) {
+        if (lane < n_seg) a.partial[row * n_seg + lane] = r0;
+        if (lane + 32 < n_seg) a.partial[row * n_seg + lane + 32] = r1;
+    }
+    float S = 0.f;
+    const int lo = n_seg < 32 ? n_seg : 32;
+    for (int j = 0; j < lo; ++j) S += __shfl_sync(0xffffffffu, r0, j);
+    for (int j = 32; j < n_seg; ++j) S += __shfl_sync(0xffffffffu, r1, j - 32);
+    __syncwarp();  // the scratch is rewritten by the next row
+    return S;
+}
+
+// Statistic of one row held in shared memory, by one warp (any width): lane
+// l adds its chunks l, l + 32, ... in order into a running pair sum that is
+// parked in the warp's scratch `part` (slot [segment][lane]) whenever a
+// segment ends; the slots are then reduced (finish_statistic or
+// finish_many) and the segments added left to right.  Returns S.
+template <typename TA, bool STATS, bool MANY = false>
 __device__ __forceinline__ float row_statistic(const Args &a, const Job &J, const uint8_t *srow, int64_t row,
                                                int lane, float *part) {
+    constexpr int STRIDE = MANY ? kManySegStride : 32;
     const int nchunks = J.nchunks;
     const int sc = J.seg_chunks;
+    if constexpr (MANY) {
+        // with 32 or more chunks per segment every lane has a chunk in every
+        // segment, so every slot is written below; otherwise clear them first
+        if (sc < 32)
+            for (int j = 0; j < a.n_seg; ++j) part[j * STRIDE + lane] = 0.f;
+    } else {
 #pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
+        for (int j = 0; j < kFastMaxSeg; ++j) part[j * 32 + lane] = 0.f;
+    }
     float2 cur = make_float2(0.f, 0.f);
     int cur_seg = 0, next_bound = sc;
     int c0 = 0;
@@ -268,18 +321,19 @@ __device__ __forceinline__ float row_statistic(const Args &a, const Job &J, cons
             } else {
 #pragma unroll
                 for (int u = 0; u < kUnroll; ++u)
-                    accumulate(sq[u], c0 + u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
+                    accumulate<STRIDE>(sq[u], c0 + u * 32 + lane, cur, cur_seg, next_bound, sc, part, lane);
             }
         }
     }
     for (; c0 < nchunks; c0 += 32) {
         const int c = c0 + lane;
         if (c < nchunks)
-            accumulate(chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)), c, cur, cur_seg,
-                       next_bound, sc, part, lane);
+            accumulate<STRIDE>(chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)), c, cur, cur_seg,
+                               next_bound, sc, part, lane);
     }
-    part[cur_seg * 32 + lane] = cur.x + cur.y;
-    return finish_statistic<STATS>(a, part, row, lane);
+    part[cur_seg * STRIDE + lane] = cur.x + cur.y;
+    if constexpr (MANY) return finish_many<STATS>(a, part, row, lane);
+    else return finish_statistic<STATS>(a, part, row, lane);
 }
 
 // Statistic of a narrow row (32 * CPL chunks, CPL <= 4) whose segments are
@@ -315,8 +369,9 @@ __device__ __forceinline__ float narrow_statistic(const uint8_t *srow, int lane,
 
 // Kernel flavours, chosen per launch from the rows' shapes so that each
 // keeps only the register budget of the paths it can take.
-constexpr int kFlavorGeneric = 0;  // any row
+constexpr int kFlavorGeneric = 0;  // any row, up to 8 segments
 constexpr int kFlavorNarrow = 1;   // some rows take the narrow statistic
+constexpr int kFlavorManySeg = 2;  // 9 .. 64 segments
 
 // One row held in shared memory, processed by one warp.  `part` is the warp's
 // [8][32] scratch for lane partials; `wsm` the job's fp32 weights.  FLAVOR
@@ -337,7 +392,7 @@ __device__ __forceinline__ void process_row(const Args &a, const Job &J, const u
             if ((lane & (lps - 1)) == 0) a.partial[row * n_seg + lane / lps] = seg;
         }
     } else {
-        S = row_statistic<TA, STATS>(a, J, srow, row, lane, part);
+        S = row_statistic<TA, STATS, FLAVOR == kFlavorManySeg>(a, J, srow, row, lane, part);
     }
 
     // ---- apply
@@ -438,7 +493,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
     const int64_t nt0 = a.job[0].ntiles;
     const int64_t step = (int64_t)W * gridDim.x;
     const int64_t first = blockIdx.x + (int64_t)warp * gridDim.x;
-    float *part = scratch + warp * kFastMaxSeg * 32;
+    float *part = scratch + warp * a.scratch_floats;
     int64_t issued = 0;  // tiles of this warp whose copies were issued
     if (lane == 0) {
         for (int j = 0; j < spw; ++j) {

@@ -1,10 +1,11 @@
 """GPU parity of the cluster path: rows spread over the CTAs of a thread-block cluster.
 
 qknorm_fused and rmsnorm_partial_stats take it for 16-byte-aligned rows with
-more than 8 segments, or wider than one CTA's registers hold (more than 65536
-bf16 / 32768 fp32 elements).  Each CTA forms the partial sums of squares of
-the segments its slice touches and the CTAs exchange only those scalars
-through distributed shared memory.  Bars as everywhere: bf16 within 1 ulp of
+more than 8 segments that the staged kernel's shared-memory ring does not
+hold (rows of more than about 40 KiB), and for rows wider than one CTA's
+registers hold (more than 65536 bf16 / 32768 fp32 elements).  Each CTA forms
+the partial sums of squares of the segments its slice touches and the CTAs
+exchange only those scalars through distributed shared memory.  Bars as everywhere: bf16 within 1 ulp of
 RNE(oracle), fp32 within 1e-5 relative, partial sums within 1e-5 relative,
 bitwise identical between runs.
 """
@@ -37,9 +38,12 @@ def _run(wl_name, T, dq, dk, n_seg, seed=0):
 
 @pytest.mark.parametrize("wl_name", ["prefill_gqa", "tiny"])
 @pytest.mark.parametrize("n_seg", [16, 64])
-def test_many_segments(cuda_lib, wl_name, n_seg):
-    # 16 and 64 segments (the fast paths stop at 8); q 4096 + k 1024, ragged token count
-    _run(wl_name, 37, 4096, 1024, n_seg, seed=n_seg)
+@pytest.mark.parametrize("dq", [4096, 32768])
+def test_many_segments(cuda_lib, wl_name, n_seg, dq):
+    # 16 and 64 segments (the register kernel stops at 8): q 4096 + k 1024 rows go
+    # through the staged kernel's many-segment statistic, q rows of 32768 (64 / 128
+    # KiB) through the cluster; ragged token count
+    _run(wl_name, 37, dq, 1024, n_seg, seed=n_seg)
 
 
 @pytest.mark.parametrize("wl_name,dq,dk,n_seg", [

@@ -287,6 +287,32 @@ def test_register_kernel_many_rows(cuda_lib, dq, dk, n_seg):
     assert_f32_close(p, oracle.segment_partials(inp["q"].cpu(), n_seg), tol=PARTIAL_REL_TOL, what="partials")
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dq,dk,n_seg", [(4096, 1024, 16), (5120, 1024, 64), (5120, 5120, 40), (2048, 256, 32),
+                                         (1024, 128, 16)])
+def test_many_segments_staged(cuda_lib, dtype, dq, dk, n_seg):
+    # 9 .. 64 segments through the staged kernel's many-segment statistic: segments of
+    # 2 chunks (lanes skip segments), a count that is not a power of two, ragged T;
+    # the partial sums themselves, and the same bits from a short launch
+    if dtype == torch.float32 and (dq // n_seg) % 4:
+        pytest.skip("segments not whole fp32 chunks")
+    T = 301
+    g = torch.Generator().manual_seed(dq + dk + n_seg)
+    q = (torch.randn(T, dq, generator=g) * 2).to(dtype).to(DEV)
+    k = torch.randn(T, dk, generator=g).to(dtype).to(DEV)
+    wq = (1 + 0.1 * torch.randn(dq, generator=g)).to(dtype).to(DEV)
+    wk = (1 + 0.1 * torch.randn(dk, generator=g)).to(dtype).to(DEV)
+    qo, ko = qk.qknorm_fused(q, k, wq, wk, 1e-6, n_seg)
+    qs, ks = qk.qknorm_fused(q[:5], k[:5], wq, wk, 1e-6, n_seg)
+    p = qk.rmsnorm_partial_stats(q, n_seg)
+    torch.cuda.synchronize()
+    check(qo, q, wq, 1e-6, f"q d={dq} n_seg={n_seg}")
+    check(ko, k, wk, 1e-6, f"k d={dk} n_seg={n_seg}")
+    bits = (lambda t: t.view(torch.int16)) if dtype == torch.bfloat16 else (lambda t: t)
+    assert torch.equal(bits(qo[:5]), bits(qs)) and torch.equal(bits(ko[:5]), bits(ks))
+    assert_f32_close(p, oracle.segment_partials(q.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials n_seg={n_seg}")
+
+
 def test_long_launch_matches_short_launch(cuda_lib):
     # batch invariance: rows normalised in a launch of 65536 + 65536 rows and in a
     # launch of a few hundred agree bit for bit

@@ -407,6 +407,37 @@ def run_qknorm(args, rank, world, local, pg):
     value = global_tokens / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
     achieved = per_set / (avg_launch_ms * 1e-3) / 1e9
+
+    # The segment partial sums on their own (rmsnorm_partial_stats of q, then
+    # of k), timed after the main region the same way: one graph, rotating sets.
+    for st in sets:
+        st["pq"] = torch.empty((my_tokens, wl.n_seg), dtype=torch.float32, device=dev)
+        st["pk"] = torch.empty((my_tokens, wl.n_seg), dtype=torch.float32, device=dev)
+
+    def stats_step(i):
+        st = sets[i % nsets]
+        qk.rmsnorm_partial_stats(st["q"], wl.n_seg, out=st["pq"])
+        qk.rmsnorm_partial_stats(st["k"], wl.n_seg, out=st["pk"])
+
+    stats_steps = min(steps, 200)
+    for i in range(3):
+        stats_step(i)
+    torch.cuda.synchronize()
+    sgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(sgraph):
+        for i in range(stats_steps):
+            stats_step(i)
+    sgraph.replay()
+    torch.cuda.synchronize()
+    s_ms, _ = time_launches(lambda _i: sgraph.replay(), 1, torch.cuda.current_stream(dev))
+    s_ms = max_over_ranks(s_ms, pg) / stats_steps
+    del sgraph
+    stats_bytes = my_tokens * (wl.dq + wl.dk) * (4 if wl.dtype == "f32" else 2) + 2 * my_tokens * wl.n_seg * 4
+    partial_stats = {"us_per_step": s_ms * 1e3, "launches_per_step": 2, "algorithmic_bytes": stats_bytes,
+                     "achieved_gbs": stats_bytes / (s_ms * 1e-3) / 1e9,
+                     "frac": stats_bytes / (s_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                     "what": "rmsnorm_partial_stats of q then of k (the per-segment sums alone), "
+                             f"{stats_steps} steps in one CUDA graph over the same rotating sets"}
     src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/rownorm_staged.cuh",
            "rmsnorm_qknorm_b200/csrc/rownorm_register.cuh", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
            "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
@@ -463,6 +494,7 @@ def run_qknorm(args, rank, world, local, pg):
                                           "replay; the mean includes the in-graph gaps between launches",
                          "peak_source": f"{pk_kind} HBM copy bandwidth",
                          "frac_of_8TBs": achieved / 8000.0},
+            "partial_stats": partial_stats,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": steps,
@@ -528,6 +560,15 @@ def run_flashnorm(args, rank, world, local, pg):
     total_ms = max_over_ranks(total_ms, pg)
     avg_gemm = max_over_ranks(statistics.mean(gemm_ms), pg)
     unf_ms = max_over_ranks(unf_ms, pg)
+    # the fold, an offline step (once per weight update): W' = diag(w) W, K-major
+    fold_out = torch.empty_like(Wf)
+    for _ in range(3):
+        qk.flashnorm_fold_weights(w, Wm, out=fold_out)
+    fold_n = 20
+    f_ms, _ = time_launches(lambda _i: qk.flashnorm_fold_weights(w, Wm, out=fold_out), fold_n, stream)
+    fold_us = max_over_ranks(f_ms, pg) / fold_n * 1e3
+    fold_bytes = 2 * Wm.numel() * Wm.element_size() + w.numel() * w.element_size()
+    del fold_out
     clk = clocks.stop(gpu_index=local) if clocks else None
     ms_per_step = total_ms / steps
     value = world * wl.M / (ms_per_step * 1e-3)
@@ -580,6 +621,11 @@ def run_flashnorm(args, rank, world, local, pg):
             "comparison": {"unfused_ms_per_step": unf_ms / steps, "fused_ms_per_step": ms_per_step,
                            "speedup_vs_unfused": (unf_ms / steps) / ms_per_step,
                            "unfused": "qknorm_fused RMSNorm writing x_hat, then torch.matmul (cuBLAS) with W"},
+            "fold": {"us_per_launch": fold_us, "algorithmic_bytes": fold_bytes,
+                     "achieved_gbs": fold_bytes / (fold_us * 1e-6) / 1e9,
+                     "frac": fold_bytes / (fold_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+                     "what": "flashnorm_fold_weights into the K-major W' (offline, once per weight update; "
+                             "timed after the main region, 20 launches)"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * steps, "clocks": clk,
         }), flush=True)
 

@@ -339,8 +339,10 @@ QKN_API qkn_status qkn_check_device(void *stream);
 /*
  * qkn_testing_arm_wait_fault -- TESTING ONLY: exercises the bounded waits
  * without faulting the GPU.  Arms a one-shot fault for the next launch of the
- * staged norm kernel made from this host thread (qknorm_fused or
- * rmsnorm_partial_stats on rows it handles): warp 0 of block 0 does not issue
+ * staged norm kernel made from this host thread (qknorm_fused on rows it
+ * handles, or rmsnorm_partial_stats with more than 8 segments on such rows;
+ * with fewer the statistics read rows without a staging ring and the hook
+ * stays armed): warp 0 of block 0 does not issue
  * the copies of its first tile, so its wait on that stage cannot complete;
  * every wait of that launch gives up after wait_ns (0 < wait_ns <= 2e9)
  * instead of 2 s, records the failure, drains and exits.  The launch's output

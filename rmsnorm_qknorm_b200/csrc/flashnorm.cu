@@ -63,21 +63,76 @@ __global__ void __launch_bounds__(256) fold_transpose_kernel(const TW *__restric
     }
 }
 
-// W [K][N] -> W^T [N][K] through a 64x64 shared tile (the projection reads
-// its weights K-major).
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ W,
+// Two bf16 of a word scaled by s in fp32 and rounded back (RNE), the same
+// rounding as the element-wise fold.
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float s) {
+    return pack_bf16x2(s * bf16lo(v), s * bf16hi(v));
+}
+
+// Row-major output with 16-byte accesses (N a multiple of 8, buffers 16-byte
+// aligned): one chunk of 8 consecutive n of one k row per thread and step.
+template <typename TW>
+__global__ void __launch_bounds__(256) fold_rowmajor_vec_kernel(const TW *__restrict__ w,
+                                                                const __nv_bfloat16 *__restrict__ W,
+                                                                __nv_bfloat16 *__restrict__ Wf,
+                                                                int64_t K, int64_t N) {
+    const int64_t cpr = N / 8, chunks = K * cpr;
+    for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x); i < chunks;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float sk = to_f32<TW>(w[i / cpr]);
+        uint4 v = __ldcs(reinterpret_cast<const uint4 *>(W) + i);
+        v = make_uint4(scale_bf16x2(v.x, sk), scale_bf16x2(v.y, sk), scale_bf16x2(v.z, sk), scale_bf16x2(v.w, sk));
+        __stcs(reinterpret_cast<uint4 *>(Wf) + i, v);
+    }
+}
+
+// W [K][N] -> W^T [N][K] (scaled by w[k] when SCALE) through a 64 x 64 tile
+// with 16-byte global accesses; K and N multiples of 8, buffers 16-byte
+// aligned.  A thread reads 8 consecutive n of one k row and parks them as 4
+// words in shared memory (rows of 33 words: a warp's stores hit 32 banks);
+// then it gathers one pair of n columns over 8 consecutive k and writes two
+// 16-byte chunks, W^T[n][k0 .. k0+7] and W^T[n+1][k0 .. k0+7] (eight threads
+// cover 128 contiguous bytes of each output row).
+template <typename TW, bool SCALE>
+__global__ void __launch_bounds__(256) transpose_tile_kernel(const TW *__restrict__ w,
+                                                             const __nv_bfloat16 *__restrict__ W,
                                                              __nv_bfloat16 *__restrict__ Wt, int64_t K, int64_t N) {
-    __shared__ __nv_bfloat16 tile[kFoldTile][kFoldTile + 2];
+    __shared__ uint32_t tile[kFoldTile][kFoldTile / 2 + 1];
     const int64_t k0 = (int64_t)blockIdx.y * kFoldTile, n0 = (int64_t)blockIdx.x * kFoldTile;
-    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
-    for (int r = ty; r < kFoldTile; r += 4) {
-        const int64_t k = k0 + r, n = n0 + tx;
-        if (k < K && n < N) tile[r][tx] = W[k * N + n];
+    const int t = threadIdx.x;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int idx = t + h * 256;
+        const int r = idx >> 3, c = idx & 7;  // tile row (k) and chunk of 8 n
+        const int64_t k = k0 + r, n = n0 + c * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (k < K && n < N) {
+            v = __ldcs(reinterpret_cast<const uint4 *>(W + k * N + n));
+            if constexpr (SCALE) {
+                const float sk = to_f32<TW>(w[k]);
+                v = make_uint4(scale_bf16x2(v.x, sk), scale_bf16x2(v.y, sk), scale_bf16x2(v.z, sk),
+                               scale_bf16x2(v.w, sk));
+            }
+        }
+        tile[r][c * 4 + 0] = v.x;
+        tile[r][c * 4 + 1] = v.y;
+        tile[r][c * 4 + 2] = v.z;
+        tile[r][c * 4 + 3] = v.w;
     }
     __syncthreads();
-    for (int r = ty; r < kFoldTile; r += 4) {
-        const int64_t n = n0 + r, k = k0 + tx;
-        if (n < N && k < K) Wt[n * K + k] = tile[tx][r];
+    const int p = t >> 3, kc = t & 7;  // pair of n columns, chunk of 8 k
+    uint32_t wd[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wd[j] = tile[kc * 8 + j][p];
+    // low halves hold column n0 + 2p, high halves column n0 + 2p + 1
+    const uint4 lo = make_uint4(__byte_perm(wd[0], wd[1], 0x5410), __byte_perm(wd[2], wd[3], 0x5410),
+                                __byte_perm(wd[4], wd[5], 0x5410), __byte_perm(wd[6], wd[7], 0x5410));
+    const uint4 hi = make_uint4(__byte_perm(wd[0], wd[1], 0x7632), __byte_perm(wd[2], wd[3], 0x7632),
+                                __byte_perm(wd[4], wd[5], 0x7632), __byte_perm(wd[6], wd[7], 0x7632));
+    const int64_t n = n0 + 2 * p, k = k0 + kc * 8;
+    if (k < K) {
+        if (n < N) __stcs(reinterpret_cast<uint4 *>(Wt + n * K + k), lo);
+        if (n + 1 < N) __stcs(reinterpret_cast<uint4 *>(Wt + (n + 1) * K + k), hi);
     }
 }
 
@@ -530,20 +585,32 @@ extern "C" QKN_API qkn_status flashnorm_fold_weights(const void *w, const void *
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const __nv_bfloat16 *Wb = static_cast<const __nv_bfloat16 *>(W);
     __nv_bfloat16 *Wo = static_cast<__nv_bfloat16 *>(W_folded);
+    const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(w);
+    const float *wf = static_cast<const float *>(w);
+    // 16-byte chunks of 8 bf16 when the layout allows (element-wise otherwise)
+    const bool vec = aligned(W, 16) && aligned(W_folded, 16) && N % 8 == 0 && (!out_k_major || K % 8 == 0);
     if (out_k_major) {
         const int64_t gx = (N + kFoldTile - 1) / kFoldTile, gy = (K + kFoldTile - 1) / kFoldTile;
         if (gx > 0x7fffffffLL || gy > 65535) return fail(QKN_ERR_SHAPE, "flashnorm_fold_weights: too large");
         dim3 grid((unsigned)gx, (unsigned)gy);
-        if (wdt == QKN_BF16)
-            fold_transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(w), Wb, Wo, K, N);
+        if (vec && wdt == QKN_BF16)
+            transpose_tile_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(wb, Wb, Wo, K, N);
+        else if (vec)
+            transpose_tile_kernel<float, true><<<grid, 256, 0, s>>>(wf, Wb, Wo, K, N);
+        else if (wdt == QKN_BF16)
+            fold_transpose_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(wb, Wb, Wo, K, N);
         else
-            fold_transpose_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float *>(w), Wb, Wo, K, N);
+            fold_transpose_kernel<float><<<grid, 256, 0, s>>>(wf, Wb, Wo, K, N);
     } else {
         const int blocks = 4 * sm_count();
-        if (wdt == QKN_BF16)
-            fold_rowmajor_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(w), Wb, Wo, K, N);
+        if (vec && wdt == QKN_BF16)
+            fold_rowmajor_vec_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(wb, Wb, Wo, K, N);
+        else if (vec)
+            fold_rowmajor_vec_kernel<float><<<blocks, 256, 0, s>>>(wf, Wb, Wo, K, N);
+        else if (wdt == QKN_BF16)
+            fold_rowmajor_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(wb, Wb, Wo, K, N);
         else
-            fold_rowmajor_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float *>(w), Wb, Wo, K, N);
+            fold_rowmajor_kernel<float><<<blocks, 256, 0, s>>>(wf, Wb, Wo, K, N);
     }
     return check_launch("flashnorm_fold_weights launch");
 }
@@ -575,9 +642,10 @@ extern "C" QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded
         if (gx > 0x7fffffffLL || gy > 65535) return fail(QKN_ERR_SHAPE, "flashnorm_proj: W_folded too large to transpose");
         cudaError_t e = cudaMallocAsync(&tmp, (size_t)(N * K * 2), s);
         if (e != cudaSuccess) return cuda_fail(e, "flashnorm_proj: K-major copy of W_folded");
-        transpose_bf16_kernel<<<dim3((unsigned)gx, (unsigned)gy), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(W_folded), static_cast<__nv_bfloat16 *>(tmp), K, N);
-        if (qkn_status st = check_launch("transpose_bf16_kernel launch")) {
+        // K, N multiples of 8 and 16-byte aligned buffers (checked above)
+        transpose_tile_kernel<__nv_bfloat16, false><<<dim3((unsigned)gx, (unsigned)gy), 256, 0, s>>>(
+            nullptr, static_cast<const __nv_bfloat16 *>(W_folded), static_cast<__nv_bfloat16 *>(tmp), K, N);
+        if (qkn_status st = check_launch("transpose_tile_kernel launch")) {
             cudaFreeAsync(tmp, s);
             return st;
         }

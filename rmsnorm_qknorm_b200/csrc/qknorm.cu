@@ -245,6 +245,29 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     return launch_staged_kernel<TA, TW, STATS, staged::kFlavorGeneric>(a, (int)grid, smem, s);
 }
 
+// rmsnorm_partial_stats on rows the staged kernel would take, up to 8
+// segments: rows read straight from global memory (rowstats_direct_kernel).
+template <typename TA>
+qkn_status launch_stats_direct(const Tensor2 &t, int64_t rows, int n_seg, float *partial, cudaStream_t s) {
+    constexpr int E = Chunk<TA>::E;
+    staged::Args a{};
+    a.njobs = 1;
+    a.n_seg = n_seg;
+    a.partial = partial;
+    staged::Job &J = a.job[0];
+    J.x = static_cast<const uint8_t *>(t.x);
+    J.ld_bytes = t.ld * (int64_t)sizeof(TA);
+    J.rows = rows;
+    J.d = (int)t.d;
+    J.row_bytes = (int)(t.d * (int64_t)sizeof(TA));
+    J.nchunks = (int)(t.d / E);
+    J.seg_chunks = J.nchunks / n_seg;
+    const int64_t need = (rows + 7) / 8, cap = 4 * (int64_t)sm_count();
+    const unsigned grid = (unsigned)(need < cap ? need : cap);
+    staged::rowstats_direct_kernel<TA><<<grid, 256, 0, s>>>(a);
+    return check_launch("rowstats_direct_kernel launch");
+}
+
 template <typename TA, typename TW, bool STATS>
 qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps,
                     float *partial, cudaStream_t s) {
@@ -293,8 +316,10 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
         int64_t w_bytes = 0;
         for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
         int warps = 0, spw = 0, sb = 0;
-        if (staged_geometry(max_row_bytes, w_bytes, n_seg, &warps, &spw, &sb))
+        if (staged_geometry(max_row_bytes, w_bytes, n_seg, &warps, &spw, &sb)) {
+            if (STATS && n_seg <= kFastMaxSeg) return launch_stats_direct<TA>(ts[0], rows, n_seg, partial, s);
             return launch_staged<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, warps, spw, sb, s);
+        }
     }
 
     if (vec) {

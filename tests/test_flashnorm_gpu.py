@@ -30,8 +30,10 @@ def _inputs(M, K, N, seed=0):
 
 
 @pytest.mark.parametrize("k_major", [True, False])
-@pytest.mark.parametrize("K,N", [(64, 64), (200, 136), (4096, 264)])
+@pytest.mark.parametrize("K,N", [(64, 64), (200, 136), (4096, 264), (13, 17), (64, 100), (20, 24)])
 def test_fold_bit_exact_bf16_weights(cuda_lib, k_major, K, N):
+    # multiples of 8 take the 16-byte tile kernels; 13 x 17, 64 x 100 (N) and
+    # 20 x 24 (K, for the K-major output) the element-wise ones
     _, w, Wm, _ = _inputs(8, K, N, seed=K + N)
     out = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV), k_major=k_major)
     torch.cuda.synchronize()
@@ -42,13 +44,15 @@ def test_fold_bit_exact_bf16_weights(cuda_lib, k_major, K, N):
     np.testing.assert_array_equal(got, ref)
 
 
-def test_fold_fp32_weights_within_one_ulp(cuda_lib):
+@pytest.mark.parametrize("k_major", [True, False])
+def test_fold_fp32_weights_within_one_ulp(cuda_lib, k_major):
     _, w, Wm, _ = _inputs(8, 256, 512, seed=1)
     w32 = (1 + 0.1 * torch.randn(256, generator=torch.Generator().manual_seed(2)))
-    out = qk.flashnorm_fold_weights(w32.to(DEV), Wm.to(DEV), k_major=True)
+    out = qk.flashnorm_fold_weights(w32.to(DEV), Wm.to(DEV), k_major=k_major)
     torch.cuda.synchronize()
     ref = oracle.round_bf16_bits(oracle.fold_weights(w32, Wm))
-    assert bf16_ulp_distance(bf16_bits(out).T, ref).max() <= 1
+    got = bf16_bits(out)
+    assert bf16_ulp_distance(got.T if k_major else got, ref).max() <= 1
 
 
 def _proj_check(M, K, N, seed=0, in_kernel_stats=False):

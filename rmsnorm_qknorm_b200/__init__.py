@@ -144,6 +144,22 @@ def _vec(t: torch.Tensor, name: str, n: int):
         raise ValueError(f"{name} must be a contiguous 1-D tensor of length {n}")
 
 
+def _out2d(t: torch.Tensor, name: str, rows: int, cols: int, dtype: torch.dtype) -> torch.Tensor:
+    """A caller-provided output: the exact shape and dtype, unit stride along the row."""
+    _cuda(t, name)
+    if t.dim() != 2 or tuple(t.shape) != (rows, cols) or t.dtype != dtype or (cols > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be a {dtype} [{rows}, {cols}] tensor with unit stride along the row")
+    return t
+
+
+def _device(ref: torch.Tensor, **tensors) -> torch.device:
+    """Every CUDA tensor of a call lives on ref's device; the call is made there."""
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device} but the call's inputs are on {ref.device}")
+    return ref.device
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -184,19 +200,21 @@ def qknorm_fused(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
         ldq_o, ldk_o = ldq, ldk
     else:
         q_out_t = q_out if q_out is not None else torch.empty((T, dq), dtype=q.dtype, device=q.device)
-        _, _, ldq_o = _rows(q_out_t, "q_out")
+        _, _, ldq_o = _rows(_out2d(q_out_t, "q_out", T, dq, q.dtype), "q_out")
         q_ptr_out = q_out_t.data_ptr()
         if k is not None:
             k_out_t = k_out if k_out is not None else torch.empty((T, dk), dtype=k.dtype, device=k.device)
-            _, _, ldk_o = _rows(k_out_t, "k_out")
+            _, _, ldk_o = _rows(_out2d(k_out_t, "k_out", T, dk, k.dtype), "k_out")
             k_ptr_out = k_out_t.data_ptr()
         else:
             k_out_t, k_ptr_out, ldk_o = None, None, 0
+    dev = _device(q, k=k, wq=wq, wk=wk if k is not None else None, q_out=q_out_t, k_out=k_out_t)
     lib = load_library()
-    st = lib.qknorm_fused(q.data_ptr(), k.data_ptr() if k is not None else None,
-                          wq.data_ptr(), wk.data_ptr() if k is not None else None,
-                          q_ptr_out, k_ptr_out, T, dq, dk, ldq, ldk, ldq_o, ldk_o,
-                          act, wdt, float(eps), int(n_seg), _stream(stream))
+    with torch.cuda.device(dev):
+        st = lib.qknorm_fused(q.data_ptr(), k.data_ptr() if k is not None else None,
+                              wq.data_ptr(), wk.data_ptr() if k is not None else None,
+                              q_ptr_out, k_ptr_out, T, dq, dk, ldq, ldk, ldq_o, ldk_o,
+                              act, wdt, float(eps), int(n_seg), _stream(stream))
     _check("qknorm_fused", st)
     return q_out_t, k_out_t
 
@@ -251,13 +269,15 @@ def qknorm_fused_host(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
     if workspace is None:
         workspace = torch.empty(HOST_WORKSPACE_BYTES, dtype=torch.uint8, device=wq.device)
     _cuda(workspace, "workspace")
+    dev = _device(wq, wk=wk if k is not None else None, workspace=workspace)
     lib = load_library()
-    st = lib.qknorm_fused_host(q.data_ptr(), k.data_ptr() if k is not None else None,
-                               wq.data_ptr(), wk.data_ptr() if k is not None else None,
-                               q_out.data_ptr(), k_out.data_ptr() if k is not None else None,
-                               T, dq, dk, act, wdt, float(eps), int(n_seg),
-                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                               _stream(stream))
+    with torch.cuda.device(dev):
+        st = lib.qknorm_fused_host(q.data_ptr(), k.data_ptr() if k is not None else None,
+                                   wq.data_ptr(), wk.data_ptr() if k is not None else None,
+                                   q_out.data_ptr(), k_out.data_ptr() if k is not None else None,
+                                   T, dq, dk, act, wdt, float(eps), int(n_seg),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
     _check("qknorm_fused_host", st)
     return q_out, (k_out if k is not None else None)
 
@@ -271,8 +291,10 @@ def rmsnorm_partial_stats(x: torch.Tensor, n_seg: int, *, out: torch.Tensor | No
         out = torch.empty((rows, n_seg), dtype=torch.float32, device=x.device)
     elif out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != (rows, n_seg):
         raise ValueError("out must be a contiguous fp32 tensor of shape [rows, n_seg]")
-    st = load_library().rmsnorm_partial_stats(x.data_ptr(), rows, d, ld, act, int(n_seg),
-                                              _cuda(out, "out").data_ptr(), _stream(stream))
+    dev = _device(x, out=_cuda(out, "out"))
+    with torch.cuda.device(dev):
+        st = load_library().rmsnorm_partial_stats(x.data_ptr(), rows, d, ld, act, int(n_seg),
+                                                  out.data_ptr(), _stream(stream))
     _check("rmsnorm_partial_stats", st)
     return out
 
@@ -290,9 +312,11 @@ def flashnorm_fold_weights(w: torch.Tensor, W: torch.Tensor, *, k_major: bool = 
         out = torch.empty(shape, dtype=torch.bfloat16, device=W.device)
     elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != torch.bfloat16:
         raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
-    st = load_library().flashnorm_fold_weights(w.data_ptr(), W.data_ptr(), _cuda(out, "out").data_ptr(),
-                                               K, N, _dtype_code(w.dtype), int(bool(k_major)),
-                                               _stream(stream))
+    dev = _device(W, w=w, out=_cuda(out, "out"))
+    with torch.cuda.device(dev):
+        st = load_library().flashnorm_fold_weights(w.data_ptr(), W.data_ptr(), out.data_ptr(),
+                                                   K, N, _dtype_code(w.dtype), int(bool(k_major)),
+                                                   _stream(stream))
     _check("flashnorm_fold_weights", st)
     return out
 
@@ -324,10 +348,12 @@ def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     elif tuple(out.shape) != (M, N) or not out.is_contiguous() or out.dtype != torch.bfloat16:
         raise ValueError("out must be a contiguous bf16 [M, N] tensor")
-    st = load_library().flashnorm_proj(
-        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, N, K, 1 if k_major else 0, float(eps),
-        inv_rms.data_ptr() if inv_rms is not None else None,
-        inv_rms_out.data_ptr() if inv_rms_out is not None else None, _stream(stream))
+    dev = _device(x, W_folded=W_folded, inv_rms=inv_rms, inv_rms_out=inv_rms_out, out=_cuda(out, "out"))
+    with torch.cuda.device(dev):
+        st = load_library().flashnorm_proj(
+            x.data_ptr(), W_folded.data_ptr(), out.data_ptr(), M, N, K, 1 if k_major else 0, float(eps),
+            inv_rms.data_ptr() if inv_rms is not None else None,
+            inv_rms_out.data_ptr() if inv_rms_out is not None else None, _stream(stream))
     _check("flashnorm_proj", st)
     return out
 
@@ -358,10 +384,12 @@ def rmsnorm_apply_partials(x: torch.Tensor, w: torch.Tensor, partial: torch.Tens
         y, ldo = x, ld
     else:
         y = out if out is not None else torch.empty((rows, d), dtype=x.dtype, device=x.device)
-        _, _, ldo = _rows(y, "out")
-    st = load_library().rmsnorm_apply_partials(
-        x.data_ptr(), w.data_ptr(), y.data_ptr(), rows, d, ld, ldo, partial.data_ptr(), int(n_part),
-        int(prs), int(ps), int(d_full), act, _dtype_code(w.dtype), float(eps), _stream(stream))
+        _, _, ldo = _rows(_out2d(y, "out", rows, d, x.dtype), "out")
+    dev = _device(x, w=w, partial=partial, out=y)
+    with torch.cuda.device(dev):
+        st = load_library().rmsnorm_apply_partials(
+            x.data_ptr(), w.data_ptr(), y.data_ptr(), rows, d, ld, ldo, partial.data_ptr(), int(n_part),
+            int(prs), int(ps), int(d_full), act, _dtype_code(w.dtype), float(eps), _stream(stream))
     _check("rmsnorm_apply_partials", st)
     return y
 
@@ -382,12 +410,20 @@ def qkv_norm_proj(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, nv:
     _vec(wk, "wk", nk)
     if nv > 0:
         _vec(wv, "wv", nv)
+    for name, t in (("wk", wk), ("wv", wv if nv > 0 else None)):
+        if t is not None and t.dtype != wq.dtype:
+            raise ValueError(f"{name} must have wq's dtype")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    st = load_library().qkv_norm_proj(
-        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, K, nq, nk, nv, wq.data_ptr(),
-        wk.data_ptr(), wv.data_ptr() if (wv is not None and nv > 0) else None, _dtype_code(wq.dtype),
-        float(eps), int(n_seg), _stream(stream))
+    elif not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    _out2d(out, "out", M, N, torch.bfloat16)
+    dev = _device(x, W_folded=W_folded, wq=wq, wk=wk, wv=wv if nv > 0 else None, out=out)
+    with torch.cuda.device(dev):
+        st = load_library().qkv_norm_proj(
+            x.data_ptr(), W_folded.data_ptr(), out.data_ptr(), M, K, nq, nk, nv, wq.data_ptr(),
+            wk.data_ptr(), wv.data_ptr() if (wv is not None and nv > 0) else None, _dtype_code(wq.dtype),
+            float(eps), int(n_seg), _stream(stream))
     _check("qkv_norm_proj", st)
     return out
 
@@ -436,16 +472,22 @@ def qkv_proj_qknorm(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, n
             raise ValueError("inv_rms_out must be fp32")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    _out2d(out, "out", M, N, torch.bfloat16)
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         _cuda(workspace, "workspace")
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    st = load_library().qkv_proj_qknorm(
-        x.data_ptr(), W_folded.data_ptr(), _cuda(out, "out").data_ptr(), M, K, nq, nk, nv,
-        wq.data_ptr(), wk.data_ptr(), _dtype_code(wq.dtype), float(eps),
-        float(eps if eps_qk is None else eps_qk),
-        inv_rms.data_ptr() if inv_rms is not None else None,
-        inv_rms_out.data_ptr() if (inv_rms is None and inv_rms_out is not None) else None,
-        ws_ptr, ws_bytes, _stream(stream))
+    dev = _device(x, W_folded=W_folded, wq=wq, wk=wk, inv_rms=inv_rms, inv_rms_out=inv_rms_out,
+                  workspace=workspace, out=out)
+    with torch.cuda.device(dev):
+        st = load_library().qkv_proj_qknorm(
+            x.data_ptr(), W_folded.data_ptr(), out.data_ptr(), M, K, nq, nk, nv,
+            wq.data_ptr(), wk.data_ptr(), _dtype_code(wq.dtype), float(eps),
+            float(eps if eps_qk is None else eps_qk),
+            inv_rms.data_ptr() if inv_rms is not None else None,
+            inv_rms_out.data_ptr() if (inv_rms is None and inv_rms_out is not None) else None,
+            ws_ptr, ws_bytes, _stream(stream))
     _check("qkv_proj_qknorm", st)
     return out

@@ -326,3 +326,30 @@ def test_long_launch_matches_short_launch(cuda_lib):
     g = torch.Generator().manual_seed(1)
     rows = torch.randint(0, 65536, (64,), generator=g).to(DEV)
     check(qo[rows], inp["q"][rows], inp["wq"], inp["eps"], "long launch q sampled")
+
+
+def test_binding_rejects_mismatched_outputs(cuda_lib):
+    # caller-provided outputs must have exactly the shape and dtype the call writes:
+    # the binding refuses them before anything is launched
+    q = torch.randn(16, 256, device=DEV).to(torch.bfloat16)
+    w = torch.ones(256, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError):
+        qk.qknorm_fused(q, None, w, None, 1e-6, 1, q_out=torch.empty(8, 256, dtype=torch.bfloat16, device=DEV))
+    with pytest.raises(ValueError):
+        qk.qknorm_fused(q, None, w, None, 1e-6, 1, q_out=torch.empty(16, 256, dtype=torch.float32, device=DEV))
+    p = qk.rmsnorm_partial_stats(q, 1)
+    with pytest.raises(ValueError):
+        qk.rmsnorm_apply_partials(q, w, p, 256, 1e-6, out=torch.empty(16, 128, dtype=torch.bfloat16, device=DEV))
+    x = torch.randn(128, 256, device=DEV).to(torch.bfloat16)
+    Wf = torch.randn(384, 256, device=DEV).to(torch.bfloat16)
+    wqk = torch.ones(128, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError):
+        qk.flashnorm_proj(x, Wf, 1e-6, out=torch.empty(128, 384, dtype=torch.float32, device=DEV))
+    with pytest.raises(ValueError):
+        qk.qkv_proj_qknorm(x, Wf, 128, 128, 128, wqk, wqk, 1e-6, out=torch.empty(128, 256, dtype=torch.bfloat16,
+                                                                                  device=DEV))
+    with pytest.raises(ValueError):
+        qk.qkv_norm_proj(x, Wf, 128, 128, 128, wqk, wqk, wqk, 1e-6, out=torch.empty(64, 384, dtype=torch.bfloat16,
+                                                                                     device=DEV))
+    torch.cuda.synchronize()
+    assert qk.load_library().qkn_check_device(None) == 0

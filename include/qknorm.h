@@ -62,7 +62,8 @@ typedef enum {
 /*
  * qknorm_fused -- layerwise QK-Norm of the query and key rows in ONE launch.
  *
- * Defined by: SwiftQK (montaan.com 2608.09160), abstract -- QK-Norm is an
+ * Defined by: "SwiftQK: Fast and Communication-Efficient Tensor Parallelism
+ * for Query-Key Normalization", abstract -- QK-Norm is an
  * RMSNorm whose factor depends on each token's full q (resp. k) vector; under
  * tensor parallelism every shard contributes a scalar partial sum of squares
  * and only these scalars are combined.  Here the n_seg shards are emulated on

@@ -503,6 +503,57 @@ def run_qknorm(args, rank, world, local, pg):
         print(json.dumps(out), flush=True)
 
 
+def host_pipeline(hx, hy, call, dev, nchunks=8):
+    """One end-to-end step from pinned host memory through the public API:
+    row chunks of x are uploaded, projected (`call(dx, dy, inv, slot)`) and
+    downloaded on three streams, one per role, so the upload of one chunk, the
+    kernel of another and the download of a third overlap.  Three buffer slots
+    rotate; events order every reuse.  The kernels run one after another on
+    their stream (the fused QKV kernel is a cooperative launch)."""
+    import torch
+    M = hx.shape[0]
+    rows = (M + nchunks - 1) // nchunks
+    s_up, s_comp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
+    slots = [(torch.empty((rows, hx.shape[1]), dtype=hx.dtype, device=dev),
+              torch.empty((rows, hy.shape[1]), dtype=hy.dtype, device=dev),
+              torch.empty(rows, dtype=torch.float32, device=dev)) for _ in range(3)]
+
+    def step(_i):
+        cur = torch.cuda.current_stream(dev)
+        start = torch.cuda.Event()
+        start.record(cur)
+        for st in (s_up, s_comp, s_down):
+            st.wait_event(start)
+        up, comp, down = [], [], []
+        for c in range(nchunks):
+            r0 = c * rows
+            n = min(rows, M - r0)
+            if n <= 0:
+                break
+            dx, dy, inv = slots[c % 3]
+            with torch.cuda.stream(s_up):
+                if c >= 3:
+                    s_up.wait_event(comp[c - 3])  # the slot's x was read
+                dx[:n].copy_(hx[r0:r0 + n], non_blocking=True)
+                up.append(torch.cuda.Event())
+                up[c].record(s_up)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(up[c])
+                if c >= 3:
+                    s_comp.wait_event(down[c - 3])  # the slot's y was downloaded
+                call(dx[:n], dy[:n], inv[:n], c % 3)
+                comp.append(torch.cuda.Event())
+                comp[c].record(s_comp)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(comp[c])
+                hy[r0:r0 + n].copy_(dy[:n], non_blocking=True)
+                down.append(torch.cuda.Event())
+                down[c].record(s_down)
+        cur.wait_event(down[-1])
+
+    return step
+
+
 def run_flashnorm(args, rank, world, local, pg):
     import torch
     import rmsnorm_qknorm_b200 as qk
@@ -582,12 +633,8 @@ def run_flashnorm(args, rank, world, local, pg):
     if args.e2e_steps > 0:
         hx = x.cpu().pin_memory()
         hy = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
-        dx = torch.empty_like(x)
-
-        def e2e_step(_i):
-            dx.copy_(hx, non_blocking=True)
-            qk.flashnorm_proj(dx, Wf, wl.eps, inv_rms_out=inv, out=y)
-            hy.copy_(y, non_blocking=True)
+        e2e_step = host_pipeline(
+            hx, hy, lambda dx, dy, dinv, _slot: qk.flashnorm_proj(dx, Wf, wl.eps, inv_rms_out=dinv, out=dy), dev)
 
         e2e_step(0)
         barrier(pg)
@@ -596,7 +643,8 @@ def run_flashnorm(args, rank, world, local, pg):
         e_ms = max_over_ranks(e_ms, pg)
         e2e = {"value": world * wl.M / (e_ms / args.e2e_steps * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2,
-               "note": "pinned host x -> device, flashnorm_proj, device -> pinned host y, per step"}
+               "note": "pinned host x -> device, flashnorm_proj, device -> pinned host y, per step, in 8 row "
+                       "chunks with upload, kernel and download overlapped on three streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -704,12 +752,13 @@ def run_qkv(args, rank, world, local, pg):
     if args.e2e_steps > 0:
         hx = x.cpu().pin_memory()
         hy = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
-        dx = torch.empty_like(x)
-
-        def e2e_step(_i):
-            dx.copy_(hx, non_blocking=True)
-            qk.qkv_proj_qknorm(dx, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms_out=inv, workspace=ws, out=y)
-            hy.copy_(y, non_blocking=True)
+        chunk_rows = (wl.M + 7) // 8
+        wss = [torch.empty(qk.qkv_proj_qknorm_workspace_bytes(chunk_rows, nq, nk, nv), dtype=torch.uint8,
+                           device=dev) for _ in range(3)]
+        e2e_step = host_pipeline(
+            hx, hy, lambda dx, dy, dinv, slot: qk.qkv_proj_qknorm(dx, Wf, nq, nk, nv, wq, wk, wl.eps,
+                                                                  inv_rms_out=dinv, workspace=wss[slot], out=dy),
+            dev)
 
         e2e_step(0)
         barrier(pg)
@@ -718,7 +767,8 @@ def run_qkv(args, rank, world, local, pg):
         e_ms = max_over_ranks(e_ms, pg)
         e2e = {"value": world * wl.M / (e_ms / args.e2e_steps * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2,
-               "note": "pinned host x -> device, qkv_proj_qknorm, device -> pinned host y, per step"}
+               "note": "pinned host x -> device, qkv_proj_qknorm, device -> pinned host y, per step, in 8 row "
+                       "chunks with upload, kernel and download overlapped on three streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

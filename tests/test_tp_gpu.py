@@ -56,6 +56,24 @@ def test_tensor_parallel_emulated_on_one_gpu(cuda_lib, shards):
         assert_bf16_close(y, oracle.rmsnorm(x.cpu(), w.cpu(), inp["eps"]), f"{shards} shards d={d}")
 
 
+def test_tensor_parallel_full_prefill_sampled(cuda_lib):
+    # the prefill GQA workload at full size split 8 ways as the tensor-parallel bench
+    # splits it (q 8 x 640, k 8 x 128): every shard's partials, combined in shard
+    # order, then each shard's apply; sampled rows against the oracle
+    inp = W.make_qknorm_inputs("prefill_gqa", seed=0, device=DEV)
+    g = torch.Generator().manual_seed(9)
+    rows = torch.randint(0, inp["q"].shape[0], (256,), generator=g).to(DEV)
+    for x, w in ((inp["q"], inp["wq"]), (inp["k"], inp["wk"])):
+        T, d = x.shape
+        s = d // 8
+        slices = [x[:, j * s:(j + 1) * s].contiguous() for j in range(8)]
+        parts = torch.stack([qk.rmsnorm_partial_stats(sl, 1)[:, 0] for sl in slices])  # [8, T]
+        y = torch.cat([qk.rmsnorm_apply_partials(slices[j], w[j * s:(j + 1) * s].contiguous(), parts.t(), d,
+                                                 inp["eps"]) for j in range(8)], dim=1)
+        torch.cuda.synchronize()
+        assert_bf16_close(y[rows], oracle.rmsnorm(x[rows].cpu(), w.cpu(), inp["eps"]), f"8 shards d={d} sampled")
+
+
 def test_apply_partials_fp32_and_unaligned(cuda_lib):
     g = torch.Generator().manual_seed(4)
     x = torch.randn(33, 100, generator=g).to(DEV)          # d not a multiple of 4: element path

@@ -419,6 +419,12 @@ def run_qknorm(args, rank, world, local, pg):
         qk.rmsnorm_partial_stats(st["q"], wl.n_seg, out=st["pq"])
         qk.rmsnorm_partial_stats(st["k"], wl.n_seg, out=st["pk"])
 
+    # the same launches made one by one from Python (no graph): what a caller
+    # without graph capture sees per launch, host launch path included
+    eager_n = min(steps, 200)
+    ev_ms, _ = time_launches(step, eager_n, stream)
+    eager_launch_us = max_over_ranks(ev_ms, pg) / eager_n * 1e3
+
     stats_steps = min(steps, 200)
     for i in range(3):
         stats_step(i)
@@ -495,6 +501,7 @@ def run_qknorm(args, rank, world, local, pg):
                          "peak_source": f"{pk_kind} HBM copy bandwidth",
                          "frac_of_8TBs": achieved / 8000.0},
             "partial_stats": partial_stats,
+            "eager_launch_us": eager_launch_us,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": steps,

@@ -133,9 +133,13 @@ def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
 
 def _rows(t: torch.Tensor, name: str):
     _cuda(t, name)
-    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+    if t.dim() != 2:
         raise ValueError(f"{name} must be 2-D with unit stride along the row")
-    return t.shape[0], t.shape[1], max(t.stride(0), t.shape[1])
+    rows, cols = t.shape
+    s0, s1 = t.stride()
+    if cols > 1 and s1 != 1:
+        raise ValueError(f"{name} must be 2-D with unit stride along the row")
+    return rows, cols, max(s0, cols)
 
 
 def _vec(t: torch.Tensor, name: str, n: int):
@@ -154,14 +158,43 @@ def _out2d(t: torch.Tensor, name: str, rows: int, cols: int, dtype: torch.dtype)
 
 def _device(ref: torch.Tensor, **tensors) -> torch.device:
     """Every CUDA tensor of a call lives on ref's device; the call is made there."""
+    dev = ref.device
     for name, t in tensors.items():
-        if t is not None and t.device != ref.device:
-            raise ValueError(f"{name} is on {t.device} but the call's inputs are on {ref.device}")
-    return ref.device
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device} but the call's inputs are on {dev}")
+    return dev
+
+
+class _On:
+    """Makes the data's device current for the library call, only when it is not."""
+
+    __slots__ = ("index", "prev")
+
+    def __init__(self, dev: torch.device):
+        self.index = dev.index
+
+    def __enter__(self):
+        self.prev = torch.cuda.current_device()
+        if self.prev != self.index:
+            torch.cuda.set_device(self.index)
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev != self.index:
+            torch.cuda.set_device(self.prev)
+        return False
+
+
+# The current stream's raw handle without building a Stream object (the
+# public route costs a few microseconds per call).
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream(stream) -> int:
+    """Handle of `stream`, or of the current device's current stream."""
     if stream is None:
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device())
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
@@ -210,7 +243,7 @@ def qknorm_fused(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
             k_out_t, k_ptr_out, ldk_o = None, None, 0
     dev = _device(q, k=k, wq=wq, wk=wk if k is not None else None, q_out=q_out_t, k_out=k_out_t)
     lib = load_library()
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = lib.qknorm_fused(q.data_ptr(), k.data_ptr() if k is not None else None,
                               wq.data_ptr(), wk.data_ptr() if k is not None else None,
                               q_ptr_out, k_ptr_out, T, dq, dk, ldq, ldk, ldq_o, ldk_o,
@@ -271,7 +304,7 @@ def qknorm_fused_host(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
     _cuda(workspace, "workspace")
     dev = _device(wq, wk=wk if k is not None else None, workspace=workspace)
     lib = load_library()
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = lib.qknorm_fused_host(q.data_ptr(), k.data_ptr() if k is not None else None,
                                    wq.data_ptr(), wk.data_ptr() if k is not None else None,
                                    q_out.data_ptr(), k_out.data_ptr() if k is not None else None,
@@ -292,7 +325,7 @@ def rmsnorm_partial_stats(x: torch.Tensor, n_seg: int, *, out: torch.Tensor | No
     elif out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != (rows, n_seg):
         raise ValueError("out must be a contiguous fp32 tensor of shape [rows, n_seg]")
     dev = _device(x, out=_cuda(out, "out"))
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = load_library().rmsnorm_partial_stats(x.data_ptr(), rows, d, ld, act, int(n_seg),
                                                   out.data_ptr(), _stream(stream))
     _check("rmsnorm_partial_stats", st)
@@ -313,7 +346,7 @@ def flashnorm_fold_weights(w: torch.Tensor, W: torch.Tensor, *, k_major: bool = 
     elif tuple(out.shape) != shape or not out.is_contiguous() or out.dtype != torch.bfloat16:
         raise ValueError(f"out must be a contiguous bf16 tensor of shape {shape}")
     dev = _device(W, w=w, out=_cuda(out, "out"))
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = load_library().flashnorm_fold_weights(w.data_ptr(), W.data_ptr(), out.data_ptr(),
                                                    K, N, _dtype_code(w.dtype), int(bool(k_major)),
                                                    _stream(stream))
@@ -349,7 +382,7 @@ def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *
     elif tuple(out.shape) != (M, N) or not out.is_contiguous() or out.dtype != torch.bfloat16:
         raise ValueError("out must be a contiguous bf16 [M, N] tensor")
     dev = _device(x, W_folded=W_folded, inv_rms=inv_rms, inv_rms_out=inv_rms_out, out=_cuda(out, "out"))
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = load_library().flashnorm_proj(
             x.data_ptr(), W_folded.data_ptr(), out.data_ptr(), M, N, K, 1 if k_major else 0, float(eps),
             inv_rms.data_ptr() if inv_rms is not None else None,
@@ -386,7 +419,7 @@ def rmsnorm_apply_partials(x: torch.Tensor, w: torch.Tensor, partial: torch.Tens
         y = out if out is not None else torch.empty((rows, d), dtype=x.dtype, device=x.device)
         _, _, ldo = _rows(_out2d(y, "out", rows, d, x.dtype), "out")
     dev = _device(x, w=w, partial=partial, out=y)
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = load_library().rmsnorm_apply_partials(
             x.data_ptr(), w.data_ptr(), y.data_ptr(), rows, d, ld, ldo, partial.data_ptr(), int(n_part),
             int(prs), int(ps), int(d_full), act, _dtype_code(w.dtype), float(eps), _stream(stream))
@@ -419,7 +452,7 @@ def qkv_norm_proj(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, nv:
         raise ValueError("out must be contiguous")
     _out2d(out, "out", M, N, torch.bfloat16)
     dev = _device(x, W_folded=W_folded, wq=wq, wk=wk, wv=wv if nv > 0 else None, out=out)
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = load_library().qkv_norm_proj(
             x.data_ptr(), W_folded.data_ptr(), out.data_ptr(), M, K, nq, nk, nv, wq.data_ptr(),
             wk.data_ptr(), wv.data_ptr() if (wv is not None and nv > 0) else None, _dtype_code(wq.dtype),
@@ -481,7 +514,7 @@ def qkv_proj_qknorm(x: torch.Tensor, W_folded: torch.Tensor, nq: int, nk: int, n
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     dev = _device(x, W_folded=W_folded, wq=wq, wk=wk, inv_rms=inv_rms, inv_rms_out=inv_rms_out,
                   workspace=workspace, out=out)
-    with torch.cuda.device(dev):
+    with _On(dev):
         st = load_library().qkv_proj_qknorm(
             x.data_ptr(), W_folded.data_ptr(), out.data_ptr(), M, K, nq, nk, nv,
             wq.data_ptr(), wk.data_ptr(), _dtype_code(wq.dtype), float(eps),

@@ -87,9 +87,9 @@ typedef enum {
  * Alignment: any element-aligned pointers and pitches are accepted.  When
  * every row start is 16-byte aligned and each segment is a whole number of
  * 16-byte chunks, a vectorised kernel runs: rows held in registers when
- * n_seg <= 8 and the widest of q and k is at most 3072 bytes (4096 for
- * rmsnorm_partial_stats); else rows staged through shared memory while the
- * widest row fits the staging ring (about 40 KiB, any n_seg); wider rows
+ * n_seg <= 8 and the widest of q and k is at most 4096 bytes; else rows
+ * staged through shared memory while the widest row fits the staging ring
+ * (about 40 KiB, any n_seg); wider rows
  * spread over the CTAs of a thread-block cluster that exchange only their
  * per-segment partial sums (rows up to 8 x 16384 bf16 / 8 x 8192 fp32
  * elements).  Otherwise a slower element-wise kernel computes the same

@@ -103,9 +103,9 @@ qkn_status launch_cluster(const Tensor2 *ts, int njobs, int64_t rows, int n_seg,
     return check_launch("rownorm_cluster_kernel launch");
 }
 
-// Widest row (bytes, over the launch's jobs) that the register kernel takes
+// Widest row (bytes, over the launch's jobs) that the register kernels take
 // although the staged kernel's ring would hold it.
-constexpr int64_t kRegisterMaxRowBytes = 3072;
+constexpr int64_t kRegisterMaxRowBytes = 4096;
 constexpr int64_t kRegisterMaxRowBytesStats = 4096;
 
 // Vector-kernel configurations, tried in order: the first whose CPT covers
@@ -127,6 +127,16 @@ qkn_status launch_vec(RowArgs &a, int njobs, cudaStream_t s) {
     if (blocks > 0x7fffffffLL) return fail(QKN_ERR_SHAPE, "too many rows for one launch");
     rownorm_vec_kernel<TA, TW, CPT, BLOCK, STATS><<<(unsigned)blocks, BLOCK, 0, s>>>(a);
     return check_launch("rownorm_vec_kernel launch");
+}
+
+template <typename TA, typename TW, bool STATS>
+qkn_status launch_vec_stream(RowArgs &a, int njobs, cudaStream_t s) {
+    int64_t groups = 0;
+    for (int i = 0; i < njobs; ++i) groups += a.job[i].nblocks;
+    const int64_t cap = 2 * (int64_t)sm_count();  // two 256-thread blocks per SM
+    const unsigned grid = (unsigned)(groups < cap ? groups : cap);
+    rownorm_vec_stream_kernel<TA, TW, STATS><<<grid, stream::BLOCK, 0, s>>>(a);
+    return check_launch("rownorm_vec_stream_kernel launch");
 }
 
 // Ring geometry for the staged kernel: stage = the widest row (rounded up to
@@ -306,8 +316,9 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
     // Narrow rows go to the register kernel: a stage of the staged kernel
     // holds one row of the launch's widest job, so rows of a few hundred bytes
     // would move in copies too small to keep HBM busy, and each warp would
-    // walk its rows one by one.  The bounds are where the two kernels measured
-    // even on B200 (rows of 1536 bf16 normalised, 2048 bf16 statistics only).
+    // walk its rows one by one.  The bound is where the kernels measured even
+    // on B200 (2048 bf16 rows: 2048 + 2048 staged 3 % ahead, 2048 + 512 and
+    // 2048 + 256 the streaming register kernel 17-23 % ahead).
     // The choice depends on the row widths alone, never on the row count.
     // More than 8 segments (the register kernel stops at 8) take the staged
     // kernel's many-segment statistic when its ring holds the rows.
@@ -341,6 +352,12 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
             J.rows_per_cta = block >> J.tpr_log2;
             J.nblocks = (rows + J.rows_per_cta - 1) / J.rows_per_cta;
         }
+        // narrow rows (at most 32 threads per row) stream through persistent
+        // blocks that load the next rows while they normalise the current ones
+        // (the statistics alone keep the one-shot form, which measured as fast
+        // or faster for them)
+        if (!STATS && cfg == 0 && max_chunks <= 32 * stream::CPT)
+            return launch_vec_stream<TA, TW, STATS>(a, njobs, s);
         if (cfg == 0) return launch_vec<TA, TW, 8, 256, STATS>(a, njobs, s);
         return launch_vec<TA, TW, 8, 1024, STATS>(a, njobs, s);
     }

@@ -176,6 +176,120 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) rownorm_vec_kernel(const 
 }
 
 // ---------------------------------------------------------------------------
+// Streaming form of the vectorised kernel for narrow rows (at most 32 threads
+// per row, CPT = 8): persistent 256-thread blocks walk the row groups
+// (rows_per_cta rows of one job) and load the next group's chunks while they
+// normalise the current one, so loads stay in flight between groups (the
+// one-shot form loads, then computes and stores with nothing in flight).  A
+// row's arithmetic -- chunk-to-thread mapping, per-thread order, butterfly
+// over the row's lanes -- is the vectorised kernel's, so the results are bit
+// for bit the same.  Warp-level only: the row's lanes are within one warp.
+namespace stream {
+
+constexpr int CPT = 8;
+constexpr int BLOCK = 256;
+
+template <typename TA>
+__device__ __forceinline__ void load_group(const RowArgs &a, int64_t g, int64_t n0, uint4 (&v)[CPT]) {
+    const int which = g >= n0 ? 1 : 0;
+    const RowJob J = pick_job(a, which);
+    const int64_t b = g - (which ? n0 : 0);
+    const int tpr = 1 << J.tpr_log2;
+    const int t = threadIdx.x & (tpr - 1);
+    const int64_t row = b * J.rows_per_cta + (threadIdx.x >> J.tpr_log2);
+    const bool active = row < J.rows;
+    const uint8_t *xr = J.x + (active ? row : 0) * J.ld_bytes;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * tpr + t;
+        if (active && c < J.nchunks) v[i] = ld_stream(xr + (int64_t)c * 16);
+        else v[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+template <typename TA, typename TW, bool STATS>
+__device__ __forceinline__ void process_group(const RowArgs &a, int64_t g, int64_t n0, const uint4 (&v)[CPT]) {
+    constexpr int E = Chunk<TA>::E;
+    const int which = g >= n0 ? 1 : 0;
+    const RowJob J = pick_job(a, which);
+    const int64_t b = g - (which ? n0 : 0);
+    const int tpr = 1 << J.tpr_log2;
+    const int t = threadIdx.x & (tpr - 1);
+    const int64_t row = b * J.rows_per_cta + (threadIdx.x >> J.tpr_log2);
+    const bool active = row < J.rows;
+    const int nchunks = J.nchunks;
+
+    float acc[kFastMaxSeg];
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) acc[j] = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * tpr + t;
+        float f[E];
+        Chunk<TA>::unpack(v[i], f);
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+        const int seg = __float2int_rz(((float)c + 0.5f) * J.inv_seg_chunks);
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j) acc[j] += (j == seg) ? s : 0.f;
+    }
+    const int n_seg = a.n_seg;
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) {
+        if (j < n_seg) {
+            for (int off = tpr >> 1; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        }
+    }
+    if constexpr (STATS) {
+        if (active && t == 0) {
+            float *p = a.partial + row * n_seg;
+#pragma unroll
+            for (int j = 0; j < kFastMaxSeg; ++j)
+                if (j < n_seg) p[j] = acc[j];
+        }
+    } else {
+        float S = 0.f;
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j)
+            if (j < n_seg) S += acc[j];
+        const float inv = rsqrtf(S / (float)J.d + a.eps);
+        uint8_t *yr = J.y + (active ? row : 0) * J.ldo_bytes;
+        const TW *w = static_cast<const TW *>(J.w);
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = i * tpr + t;
+            if (active && c < nchunks) {
+                float f[E], wf[E];
+                Chunk<TA>::unpack_again(v[i], f);
+                load_weights<TW, E>(w + (int64_t)c * E, wf);
+#pragma unroll
+                for (int e = 0; e < E; ++e) f[e] = (f[e] * inv) * wf[e];
+                st_stream(yr + (int64_t)c * 16, Chunk<TA>::pack(f));
+            }
+        }
+    }
+}
+
+}  // namespace stream
+
+template <typename TA, typename TW, bool STATS>
+__global__ void __launch_bounds__(stream::BLOCK, 2) rownorm_vec_stream_kernel(const RowArgs a) {
+    const int64_t n0 = a.job[0].nblocks, total = n0 + a.job[1].nblocks;
+    int64_t g = blockIdx.x;
+    if (g >= total) return;  // the whole block: no block-level synchronisation below
+    uint4 cur[stream::CPT], nxt[stream::CPT];
+    stream::load_group<TA>(a, g, n0, cur);
+    for (; g < total; g += gridDim.x) {
+        const int64_t gn = g + gridDim.x;
+        if (gn < total) stream::load_group<TA>(a, gn, n0, nxt);
+        stream::process_group<TA, TW, STATS>(a, g, n0, cur);
+#pragma unroll
+        for (int i = 0; i < stream::CPT; ++i) cur[i] = nxt[i];
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Element-wise kernel for any alignment, width and n_seg <= QKN_MAX_SEG: one
 // row per 256-thread block; each segment is reduced over the block in turn.
 // The row is read a second time (from L2) for the apply step.

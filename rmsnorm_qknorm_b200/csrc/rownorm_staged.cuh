@@ -12,8 +12,8 @@ namespace qkn {
 
 // ---------------------------------------------------------------------------
 // Staged kernel (rows up to ~40 KiB): persistent, one block per SM.  Launches
-// whose widest row is at most 3 KiB (4 KiB for statistics alone) take the
-// register kernel instead (qknorm.cu's dispatch).
+// whose widest row is at most 4 KiB take the register kernels instead
+// (qknorm.cu's dispatch).
 //
 // Rows reach shared memory through 1-D bulk copies (cp.async.bulk, completion
 // counted on an mbarrier per stage), so the loads in flight do not depend on

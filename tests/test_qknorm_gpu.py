@@ -269,9 +269,11 @@ def test_narrow_rows(cuda_lib, dtype, d, n_seg):
     assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials d={d}")
 
 
-@pytest.mark.parametrize("dq,dk,n_seg", [(128, 128, 1), (640, 128, 1), (1536, 256, 8), (1024, 1024, 4)])
+@pytest.mark.parametrize("dq,dk,n_seg", [(128, 128, 1), (640, 128, 1), (1536, 256, 8), (1024, 1024, 4),
+                                         (2048, 512, 2)])
 def test_register_kernel_many_rows(cuda_lib, dq, dk, n_seg):
-    # rows up to 3072 bytes (both tensors) are held in registers: several CTAs and a
+    # rows up to 4096 bytes (both tensors) are held in registers (normalised by
+    # persistent blocks that stream the rows, several groups per block): many groups, a
     # ragged last one; the first rows again in a short launch give the same bits; the
     # statistics alone (register kernel up to 4096-byte rows) against the oracle
     T = 3001
@@ -311,6 +313,23 @@ def test_many_segments_staged(cuda_lib, dtype, dq, dk, n_seg):
     bits = (lambda t: t.view(torch.int16)) if dtype == torch.bfloat16 else (lambda t: t)
     assert torch.equal(bits(qo[:5]), bits(qs)) and torch.equal(bits(ko[:5]), bits(ks))
     assert_f32_close(p, oracle.segment_partials(q.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials n_seg={n_seg}")
+
+
+@pytest.mark.parametrize("T,dq,dk", [(50001, 128, 128), (20001, 1024, 1024), (10001, 2048, 512)])
+def test_register_stream_many_groups(cuda_lib, T, dq, dk):
+    # enough rows that each persistent block of the streaming register kernel walks
+    # several row groups (loading the next while normalising the current), across
+    # the q / k job boundary; sampled rows against the oracle, a short launch bitwise
+    inp = W.make_qknorm_inputs("prefill_gqa", seed=T, device=DEV, tokens=T, dq=dq, dk=dk)
+    qo, ko = qk.qknorm_fused(inp["q"], inp["k"], inp["wq"], inp["wk"], inp["eps"], 4)
+    qs, ks = qk.qknorm_fused(inp["q"][-300:], inp["k"][-300:], inp["wq"], inp["wk"], inp["eps"], 4)
+    torch.cuda.synchronize()
+    g = torch.Generator().manual_seed(T)
+    rows = torch.cat([torch.randint(0, T, (500,), generator=g), torch.arange(T - 40, T)]).to(DEV)
+    check(qo[rows], inp["q"][rows], inp["wq"], inp["eps"], f"q T={T} d={dq}")
+    check(ko[rows], inp["k"][rows], inp["wk"], inp["eps"], f"k T={T} d={dk}")
+    assert torch.equal(qo[-300:].view(torch.int16), qs.view(torch.int16))
+    assert torch.equal(ko[-300:].view(torch.int16), ks.view(torch.int16))
 
 
 def test_long_launch_matches_short_launch(cuda_lib):

@@ -356,11 +356,16 @@ def flashnorm_fold_weights(w: torch.Tensor, W: torch.Tensor, *, k_major: bool = 
 
 def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *,
                    inv_rms: torch.Tensor | None = None, inv_rms_out: torch.Tensor | None = None,
-                   out: torch.Tensor | None = None, k_major: bool = True, stream=None) -> torch.Tensor:
+                   out: torch.Tensor | None = None, k_major: bool = True, in_kernel_stats: bool = False,
+                   stream=None) -> torch.Tensor:
     """y [M, N] = (x [M, K] @ W') * 1/rms(x), bf16 in/out, fp32 accumulate.
 
     W_folded is [N, K] (``k_major=True``, the layout the tensor cores read) or
-    [K, N] (``k_major=False``: copied K-major inside the call first).
+    [K, N] (``k_major=False``: copied K-major inside the call first).  Without
+    ``inv_rms`` the row statistics run as a separate pass overlapped with the
+    projection, into ``inv_rms_out`` (allocated here when not given);
+    ``in_kernel_stats=True`` computes them inside the projection kernel
+    instead (no [M] workspace, slower).
     """
     _cuda(x, "x")
     _cuda(W_folded, "W_folded")
@@ -377,6 +382,8 @@ def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *
             _vec(t, name, M)
             if t.dtype != torch.float32:
                 raise ValueError(f"{name} must be fp32")
+    if inv_rms is None and inv_rms_out is None and not in_kernel_stats:
+        inv_rms_out = torch.empty(M, dtype=torch.float32, device=x.device)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     elif tuple(out.shape) != (M, N) or not out.is_contiguous() or out.dtype != torch.bfloat16:

@@ -60,7 +60,7 @@ def _proj_check(M, K, N, seed=0, in_kernel_stats=False):
     xd = x.to(DEV)
     Wf = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV), k_major=True)
     if in_kernel_stats:
-        y = qk.flashnorm_proj(xd, Wf, eps)  # 1/rms computed inside the projection kernel
+        y = qk.flashnorm_proj(xd, Wf, eps, in_kernel_stats=True)  # 1/rms computed inside the projection kernel
     else:
         inv_out = torch.empty(M, dtype=torch.float32, device=DEV)
         y = qk.flashnorm_proj(xd, Wf, eps, inv_rms_out=inv_out)  # separate statistics pass
@@ -92,13 +92,26 @@ def test_proj_statistics_paths_agree(cuda_lib):
     x, w, Wm, eps = _inputs(256, 1024, 512, seed=9)
     xd = x.to(DEV)
     Wf = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV))
-    y1 = qk.flashnorm_proj(xd, Wf, eps)
+    y1 = qk.flashnorm_proj(xd, Wf, eps, in_kernel_stats=True)
     inv = torch.empty(256, dtype=torch.float32, device=DEV)
     y2 = qk.flashnorm_proj(xd, Wf, eps, inv_rms_out=inv)
     y3 = qk.flashnorm_proj(xd, Wf, eps, inv_rms=inv)
     torch.cuda.synchronize()
     assert bf16_ulp_distance(bf16_bits(y1), bf16_bits(y2)).max() <= 1
     assert torch.equal(y2.view(torch.int16), y3.view(torch.int16))
+
+
+def test_proj_default_is_the_separate_pass(cuda_lib):
+    # without inv_rms / inv_rms_out the binding supplies the workspace itself, so the
+    # default call is the separate statistics pass, bit for bit
+    x, w, Wm, eps = _inputs(300, 512, 264, seed=12)
+    xd = x.to(DEV)
+    Wf = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV))
+    inv = torch.empty(300, dtype=torch.float32, device=DEV)
+    a = qk.flashnorm_proj(xd, Wf, eps)
+    b = qk.flashnorm_proj(xd, Wf, eps, inv_rms_out=inv)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
 def test_proj_with_unit_scale_is_plain_gemm(cuda_lib):
@@ -118,7 +131,7 @@ def test_proj_deterministic(cuda_lib):
     xd = x.to(DEV)
     Wf = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV))
     inv = torch.empty(512, dtype=torch.float32, device=DEV)
-    for kw in ({}, {"inv_rms_out": inv}):
+    for kw in ({"in_kernel_stats": True}, {"inv_rms_out": inv}, {}):
         a = qk.flashnorm_proj(xd, Wf, eps, **kw)
         b = qk.flashnorm_proj(xd, Wf, eps, **kw)
         torch.cuda.synchronize()
@@ -133,7 +146,7 @@ def test_proj_full_size_sampled(cuda_lib):
     Wf = qk.flashnorm_fold_weights(inp["w"], inp["W"])
     inv = torch.empty(wl.M, dtype=torch.float32, device=DEV)
     y = qk.flashnorm_proj(inp["x"], Wf, wl.eps, inv_rms_out=inv)  # the benchmark's form
-    y_in = qk.flashnorm_proj(inp["x"], Wf, wl.eps)                # 1/rms inside the kernel
+    y_in = qk.flashnorm_proj(inp["x"], Wf, wl.eps, in_kernel_stats=True)  # 1/rms inside the kernel
     torch.cuda.synchronize()
     assert bf16_ulp_distance(bf16_bits(y_in), bf16_bits(y)).max() <= 1
     g = torch.Generator().manual_seed(3)
@@ -162,7 +175,7 @@ def test_row_major_folded_weights(cuda_lib, in_kernel_stats):
     xd = x.to(DEV)
     Wk = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV), k_major=True)
     Wr = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV), k_major=False)
-    kw = {} if in_kernel_stats else {"inv_rms_out": torch.empty(M, dtype=torch.float32, device=DEV)}
+    kw = {"in_kernel_stats": True} if in_kernel_stats else {"inv_rms_out": torch.empty(M, dtype=torch.float32, device=DEV)}
     a = qk.flashnorm_proj(xd, Wk, eps, **kw)
     b = qk.flashnorm_proj(xd, Wr, eps, k_major=False, **kw)
     torch.cuda.synchronize()

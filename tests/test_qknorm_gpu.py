@@ -332,6 +332,28 @@ def test_register_stream_many_groups(cuda_lib, T, dq, dk):
     assert torch.equal(ko[-300:].view(torch.int16), ks.view(torch.int16))
 
 
+@pytest.mark.parametrize("act,wdt", [(torch.float32, torch.float32), (torch.bfloat16, torch.float32),
+                                     (torch.float32, torch.bfloat16)])
+def test_register_stream_in_place_and_dtypes(cuda_lib, act, wdt):
+    # the streaming register kernel in place (each row read and written by its own
+    # threads, the next rows already loading) and with every dtype pairing
+    T, dq, dk = 40000, 512, 128
+    g = torch.Generator().manual_seed(17)
+    q = (torch.randn(T, dq, generator=g) * 3).to(act).to(DEV)
+    k = torch.randn(T, dk, generator=g).to(act).to(DEV)
+    wq = (1 + 0.1 * torch.randn(dq, generator=g)).to(wdt).to(DEV)
+    wk = (1 + 0.1 * torch.randn(dk, generator=g)).to(wdt).to(DEV)
+    qo, ko = qk.qknorm_fused(q, k, wq, wk, 1e-6, 2)
+    q2, k2 = q.clone(), k.clone()
+    qk.qknorm_fused(q2, k2, wq, wk, 1e-6, 2, inplace=True)
+    torch.cuda.synchronize()
+    bits = (lambda t: t.view(torch.int16)) if act == torch.bfloat16 else (lambda t: t.view(torch.int32))
+    assert torch.equal(bits(qo), bits(q2)) and torch.equal(bits(ko), bits(k2))
+    rows = torch.randint(0, T, (300,), generator=g).to(DEV)
+    check(qo[rows], q[rows], wq, 1e-6, "q sampled")
+    check(ko[rows], k[rows], wk, 1e-6, "k sampled")
+
+
 def test_long_launch_matches_short_launch(cuda_lib):
     # batch invariance: rows normalised in a launch of 65536 + 65536 rows and in a
     # launch of a few hundred agree bit for bit

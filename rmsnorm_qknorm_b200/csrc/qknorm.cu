@@ -255,8 +255,8 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     return launch_staged_kernel<TA, TW, STATS, staged::kFlavorGeneric>(a, (int)grid, smem, s);
 }
 
-// rmsnorm_partial_stats on rows the staged kernel would take, up to 8
-// segments: rows read straight from global memory (rowstats_direct_kernel).
+// rmsnorm_partial_stats on rows the staged kernel would take: rows read
+// straight from global memory (rowstats_direct_kernel).
 template <typename TA>
 qkn_status launch_stats_direct(const Tensor2 &t, int64_t rows, int n_seg, float *partial, cudaStream_t s) {
     constexpr int E = Chunk<TA>::E;
@@ -272,9 +272,28 @@ qkn_status launch_stats_direct(const Tensor2 &t, int64_t rows, int n_seg, float 
     J.row_bytes = (int)(t.d * (int64_t)sizeof(TA));
     J.nchunks = (int)(t.d / E);
     J.seg_chunks = J.nchunks / n_seg;
+    a.scratch_floats = staged::scratch_floats(n_seg);
     const int64_t need = (rows + 7) / 8, cap = 4 * (int64_t)sm_count();
     const unsigned grid = (unsigned)(need < cap ? need : cap);
-    staged::rowstats_direct_kernel<TA><<<grid, 256, 0, s>>>(a);
+    if (n_seg <= kFastMaxSeg) {
+        staged::rowstats_direct_kernel<TA, false><<<grid, 256, 0, s>>>(a);
+    } else {
+        // up to 64 slots of 33 floats per warp: at most 8 warps x 8448 bytes,
+        // above the default 48 KiB, so the cap is raised once per device
+        const int smem = 8 * a.scratch_floats * 4;
+        static std::atomic<bool> attr_set[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const bool known = dev >= 0 && dev < 64;
+        if (!known || !attr_set[dev].load(std::memory_order_acquire)) {
+            const cudaError_t e = cudaFuncSetAttribute(staged::rowstats_direct_kernel<TA, true>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       8 * staged::scratch_floats(QKN_MAX_SEG) * 4);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(rowstats_direct_kernel)");
+            if (known) attr_set[dev].store(true, std::memory_order_release);
+        }
+        staged::rowstats_direct_kernel<TA, true><<<grid, 256, smem, s>>>(a);
+    }
     return check_launch("rowstats_direct_kernel launch");
 }
 
@@ -328,7 +347,7 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
         for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
         int warps = 0, spw = 0, sb = 0;
         if (staged_geometry(max_row_bytes, w_bytes, n_seg, &warps, &spw, &sb)) {
-            if (STATS && n_seg <= kFastMaxSeg) return launch_stats_direct<TA>(ts[0], rows, n_seg, partial, s);
+            if (STATS) return launch_stats_direct<TA>(ts[0], rows, n_seg, partial, s);
             return launch_staged<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, warps, spw, sb, s);
         }
     }

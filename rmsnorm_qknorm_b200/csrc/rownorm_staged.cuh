@@ -578,21 +578,25 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
         mbar_wait(smem_u32(&full[warp * spw + (int)(k % spw)]), (uint32_t)(k / spw) & 1u, &g_norm_error, a.wait_ns);
 }
 
-// Statistics alone (rmsnorm_partial_stats with up to 8 segments, on rows the
-// staged kernel would take).  Without an apply pass a row is read once, so
+// Statistics alone (rmsnorm_partial_stats on rows the staged kernel would
+// take).  Without an apply pass a row is read once, so
 // the staging ring buys nothing: one warp per row reads it straight from
 // global memory through the same row_statistic (the same summation order,
 // hence bit for bit the partials qknorm_fused forms), with four 8-warp blocks
 // per SM for the loads in flight.  Measured on B200 against the staged form:
 // 65536 x 4096 bf16 125 -> 105 us, 16384 x 5120 44.5 -> 41.8 us.
-template <typename TA>
+// With more than 8 segments (MANY) the warps' slots live in dynamic shared
+// memory (a.scratch_floats per warp) and the many-segment statistic runs.
+template <typename TA, bool MANY>
 __global__ void __launch_bounds__(256, 4) rowstats_direct_kernel(const Args a) {
     __shared__ float scratch[8][kFastMaxSeg * 32];
+    extern __shared__ float many_scratch[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *part = MANY ? many_scratch + warp * a.scratch_floats : scratch[warp];
     const Job J = a.job[0];
     const int64_t nw = (int64_t)gridDim.x * 8;
     for (int64_t row = (int64_t)blockIdx.x * 8 + warp; row < J.rows; row += nw)
-        row_statistic<TA, true>(a, J, J.x + row * J.ld_bytes, row, lane, scratch[warp]);
+        row_statistic<TA, true, MANY>(a, J, J.x + row * J.ld_bytes, row, lane, part);
 }
 
 }  // namespace staged

@@ -41,6 +41,19 @@ def test_apply_partials_reproduces_fused(cuda_lib, name, tokens):
                            y.view(torch.int16) if y.dtype == torch.bfloat16 else y.view(torch.int32))
 
 
+@pytest.mark.parametrize("n_seg", [16, 64])
+def test_apply_partials_reproduces_fused_many_segments(cuda_lib, n_seg):
+    # with more than 8 segments too: the statistics-only partials are bit for bit
+    # the ones qknorm_fused combines (the same many-segment statistic)
+    inp = W.make_qknorm_inputs("prefill_gqa", seed=n_seg, device=DEV, tokens=200)
+    qo, ko = qk.qknorm_fused(inp["q"], inp["k"], inp["wq"], inp["wk"], inp["eps"], n_seg)
+    for x, w, y in ((inp["q"], inp["wq"], qo), (inp["k"], inp["wk"], ko)):
+        p = qk.rmsnorm_partial_stats(x, n_seg)
+        y2 = qk.rmsnorm_apply_partials(x, w, p, x.shape[1], inp["eps"])
+        torch.cuda.synchronize()
+        assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+
+
 @pytest.mark.parametrize("shards", [2, 4, 8])
 def test_tensor_parallel_emulated_on_one_gpu(cuda_lib, shards):
     inp = W.make_qknorm_inputs("prefill_gqa", seed=2, device=DEV, tokens=129)

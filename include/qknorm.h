@@ -140,7 +140,10 @@ QKN_API qkn_status qknorm_fused_host(const void *q, const void *k,
  * partial  [rows][n_seg] fp32, contiguous, written completely
  * n_seg    1 .. QKN_MAX_SEG, d % n_seg == 0
  * The summation order inside a segment is fixed for a given row width and
- * n_seg, so repeated calls give bitwise-equal partials.
+ * n_seg, so repeated calls give bitwise-equal partials; on rows wider than
+ * 4096 bytes (and up to about 40 KiB) they are bit for bit the partials
+ * qknorm_fused combines for the same rows and n_seg, so
+ * rmsnorm_apply_partials on them reproduces qknorm_fused exactly.
  */
 QKN_API qkn_status rmsnorm_partial_stats(const void *x, int64_t rows, int64_t d,
                                          int64_t ld, qkn_dtype act, int n_seg,

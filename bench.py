@@ -53,7 +53,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=None, help="timed steps (default depends on workload)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=QK_DEFAULT,
-                    choices=["tiny", "decode", "prefill_gqa", "long_context", "flashnorm_proj",
+                    choices=["tiny", "decode", "prefill_gqa", "long_context", "narrow_rows", "flashnorm_proj",
                              "qkv_proj_qknorm", "tp_qknorm"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -447,7 +447,10 @@ def run_qknorm(args, rank, world, local, pg):
     src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/rownorm_staged.cuh",
            "rmsnorm_qknorm_b200/csrc/rownorm_register.cuh", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
            "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
-    traffic = traffic_for("rownorm_staged_kernel", wl.name, src) if args.tokens is None else None
+    # the kernel the library picks for these rows (the choice depends on the widths only)
+    row_bytes = max(wl.dq, wl.dk) * (4 if wl.dtype == "f32" else 2)
+    kernel = "rownorm_vec_stream_kernel" if row_bytes <= 4096 and wl.n_seg <= 8 else "rownorm_staged_kernel"
+    traffic = traffic_for(kernel, wl.name, src) if args.tokens is None else None
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -493,7 +496,7 @@ def run_qknorm(args, rank, world, local, pg):
                               f"{nsets} rotating input sets totalling {nsets * per_set / 1e6:.0f} MB > L2")},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
-                         "kernel": "rownorm_staged_kernel",
+                         "kernel": kernel,
                          "algorithmic_bytes_per_launch": per_set,
                          "avg_launch_us": avg_launch_ms * 1e3,
                          "launch_timing": "one CUDA graph of all timed launches, CUDA events around its "

@@ -90,6 +90,10 @@ QKNORM_WORKLOADS = {
         QKNormWorkload("long_context", 131072, 4096, 4096, "bf16", 8, 1e-6, 2.0, "token_scale",
                        "Long-context QK-Norm: 131072 tokens, q/k dim 4096, bf16, per-token "
                        "log-uniform scale in [0.1, 10], n_seg=8"),
+        # not one of the stated configurations: rows narrow enough to be held in
+        # registers (a small model's q and k, 8 heads x 128), measured beside them
+        QKNormWorkload("narrow_rows", 131072, 1024, 1024, "bf16", 4, 1e-6, 1.0, "normal",
+                       "Narrow-row QK-Norm: 131072 tokens, q/k dim 1024 (8x128), bf16, n_seg=4"),
     ]
 }
 

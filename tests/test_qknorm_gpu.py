@@ -46,7 +46,7 @@ def to_dev(inp):
 
 
 @pytest.mark.parametrize("name,tokens", [("tiny", None), ("decode", None), ("prefill_gqa", 203),
-                                         ("long_context", 301)])
+                                         ("long_context", 301), ("narrow_rows", 3001)])
 def test_workload_parity_oracle_sized(cuda_lib, name, tokens):
     inp = to_dev(W.make_qknorm_inputs(name, seed=0, tokens=tokens))
     qo, ko = run_pair(inp)
@@ -79,7 +79,7 @@ def _full_size_sampled(name, n_sample=384):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["prefill_gqa", "long_context"])
+@pytest.mark.parametrize("name", ["prefill_gqa", "long_context", "narrow_rows"])
 def test_workload_parity_full_size(cuda_lib, name):
     _full_size_sampled(name)
 

@@ -630,6 +630,13 @@ def run_flashnorm(args, rank, world, local, pg):
     fold_us = max_over_ranks(f_ms, pg) / fold_n * 1e3
     fold_bytes = 2 * Wm.numel() * Wm.element_size() + w.numel() * w.element_size()
     del fold_out
+    # the row statistic on its own (the pass the step overlaps with the projection)
+    inv_alone = torch.empty_like(inv)
+    for _ in range(3):
+        qk.flashnorm_inv_rms(x, wl.eps, out=inv_alone)
+    s_ms, _ = time_launches(lambda _i: qk.flashnorm_inv_rms(x, wl.eps, out=inv_alone), fold_n, stream)
+    stats_us = max_over_ranks(s_ms, pg) / fold_n * 1e3
+    stats_bytes = x.numel() * x.element_size() + inv.numel() * 4
     clk = clocks.stop(gpu_index=local) if clocks else None
     ms_per_step = total_ms / steps
     value = world * wl.M / (ms_per_step * 1e-3)
@@ -679,6 +686,11 @@ def run_flashnorm(args, rank, world, local, pg):
             "comparison": {"unfused_ms_per_step": unf_ms / steps, "fused_ms_per_step": ms_per_step,
                            "speedup_vs_unfused": (unf_ms / steps) / ms_per_step,
                            "unfused": "qknorm_fused RMSNorm writing x_hat, then torch.matmul (cuBLAS) with W"},
+            "inv_rms": {"us_per_launch": stats_us, "algorithmic_bytes": stats_bytes,
+                        "achieved_gbs": stats_bytes / (stats_us * 1e-6) / 1e9,
+                        "frac": stats_bytes / (stats_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+                        "what": "flashnorm_inv_rms alone (x read once, 1/rms written), 20 launches after the "
+                                "main region; in the step it runs beside the projection"},
             "fold": {"us_per_launch": fold_us, "algorithmic_bytes": fold_bytes,
                      "achieved_gbs": fold_bytes / (fold_us * 1e-6) / 1e9,
                      "frac": fold_bytes / (fold_us * 1e-6) / 1e9 / pk["hbm_gbs"],

@@ -150,6 +150,22 @@ QKN_API qkn_status rmsnorm_partial_stats(const void *x, int64_t rows, int64_t d,
                                          float *partial, void *stream);
 
 /*
+ * flashnorm_inv_rms -- FlashNorm's row statistic on its own.
+ *
+ * Defined by: FlashNorm (Graef, arXiv 2024), abstract, item (ii): the scalar
+ * 1/rms of each row, which the projection applies to its output:
+ *   inv[m] = 1 / sqrt(sum_k x[m][k]^2 / K + eps)   (fp32 sums of the bf16 x)
+ * This is the pass flashnorm_proj runs beside the projection when given
+ * inv_rms_out; the values are bit for bit the ones it writes there.
+ *
+ * x    [M][K] bf16, contiguous, 16-byte aligned; K a multiple of 8
+ * inv  [M] fp32, written completely
+ * eps  >= 0 and finite
+ */
+QKN_API qkn_status flashnorm_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float eps,
+                                     void *stream);
+
+/*
  * rmsnorm_apply_partials -- the apply step of tensor-parallel QK-Norm.
  *
  * Defined by: SwiftQK, abstract -- under tensor parallelism each shard holds

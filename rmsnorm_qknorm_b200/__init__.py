@@ -39,6 +39,7 @@ __all__ = [
     "rmsnorm_partial_stats",
     "flashnorm_fold_weights",
     "flashnorm_proj",
+    "flashnorm_inv_rms",
     "rmsnorm_apply_partials",
     "qkv_norm_proj",
     "STATUS_NAMES",
@@ -97,9 +98,10 @@ def load_library() -> ctypes.CDLL:
                                         p, ctypes.c_size_t, p]
         lib.qkv_proj_qknorm_workspace_bytes.argtypes = [i64, i64, i64, i64]
         lib.qkv_proj_qknorm_workspace_bytes.restype = ctypes.c_size_t
+        lib.flashnorm_inv_rms.argtypes = [p, p, i64, i64, f32, p]
         lib.qkn_check_device.argtypes = [p]
         for f in ("qknorm_fused", "qknorm_fused_host", "qkv_proj_qknorm", "rmsnorm_partial_stats", "flashnorm_fold_weights",
-                  "flashnorm_proj", "rmsnorm_apply_partials", "qkv_norm_proj", "qkn_check_device"):
+                  "flashnorm_proj", "flashnorm_inv_rms", "rmsnorm_apply_partials", "qkv_norm_proj", "qkn_check_device"):
             getattr(lib, f).restype = ctypes.c_int
         lib.qkn_last_error.restype = ctypes.c_char_p
         lib.qkn_last_error.argtypes = []
@@ -395,6 +397,26 @@ def flashnorm_proj(x: torch.Tensor, W_folded: torch.Tensor, eps: float = 1e-6, *
             inv_rms.data_ptr() if inv_rms is not None else None,
             inv_rms_out.data_ptr() if inv_rms_out is not None else None, _stream(stream))
     _check("flashnorm_proj", st)
+    return out
+
+
+def flashnorm_inv_rms(x: torch.Tensor, eps: float = 1e-6, *, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """FlashNorm's row statistic: fp32 [M] 1/rms of the rows of bf16 x [M, K]."""
+    _cuda(x, "x")
+    if x.dim() != 2 or not x.is_contiguous() or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a contiguous bf16 [M, K] tensor")
+    M, K = x.shape
+    if out is None:
+        out = torch.empty(M, dtype=torch.float32, device=x.device)
+    else:
+        _vec(out, "out", M)
+        if out.dtype != torch.float32:
+            raise ValueError("out must be fp32")
+    dev = _device(x, out=out)
+    with _On(dev):
+        st = load_library().flashnorm_inv_rms(x.data_ptr(), out.data_ptr(), M, K, float(eps), _stream(stream))
+    _check("flashnorm_inv_rms", st)
     return out
 
 

@@ -135,6 +135,17 @@ def test_proj_validation(lib):
     assert "16-byte" in lib.qkn_last_error().decode()
 
 
+def test_inv_rms_validation(lib):
+    f = lib.flashnorm_inv_rms
+    assert f(None, P, 4, 64, 1e-6, None) == NULL
+    assert f(P, None, 4, 64, 1e-6, None) == NULL
+    assert f(P, P, -1, 64, 1e-6, None) == SHAPE
+    assert f(P, P, 4, 60, 1e-6, None) == SHAPE     # K % 8
+    assert f(P, P, 4, 64, -1.0, None) == EPS
+    assert f(P + 8, P, 4, 64, 1e-6, None) == ALIGN  # 16-byte rows
+    assert f(None, None, 0, 64, 1e-6, None) == OK   # nothing to do: pointers unused
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
     x = torch.zeros(4, 64, dtype=torch.bfloat16)

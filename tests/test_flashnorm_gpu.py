@@ -114,6 +114,21 @@ def test_proj_default_is_the_separate_pass(cuda_lib):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("M,K", [(1, 8), (300, 4096), (1029, 1000)])
+def test_inv_rms_alone(cuda_lib, M, K):
+    # FlashNorm's row statistic on its own: within 1e-5 of the oracle, and bit for
+    # bit the values the projection writes to inv_rms_out
+    x, w, Wm, eps = _inputs(M, K, 64, seed=M + K)
+    xd = x.to(DEV)
+    inv = qk.flashnorm_inv_rms(xd, eps)
+    Wf = qk.flashnorm_fold_weights(w.to(DEV), Wm.to(DEV))
+    inv_out = torch.empty(M, dtype=torch.float32, device=DEV)
+    qk.flashnorm_proj(xd, Wf, eps, inv_rms_out=inv_out)
+    torch.cuda.synchronize()
+    assert_f32_close(inv, oracle.inv_rms(x, eps), what="inv_rms")
+    assert torch.equal(inv, inv_out)
+
+
 def test_proj_with_unit_scale_is_plain_gemm(cuda_lib):
     # a given 1/rms of 1 turns the kernel into y = x W'^T (W' = W^T for w = 1): the GEMM alone
     M, K, N = 256, 512, 768

@@ -763,6 +763,14 @@ def run_qkv(args, rank, world, local, pg):
         tot[key] = max_over_ranks(tot[key], pg)
     avg_gemm = max_over_ranks(statistics.mean(gemm_ms), pg)
     clk = clocks.stop(gpu_index=local) if clocks else None
+    # the RMSNorm-elimination form (qkv_norm_proj: the projection without the
+    # input norm, then each group's RMSNorm), timed after the main region
+    wv = torch.ones(nv, dtype=torch.bfloat16, device=dev)
+    elim = lambda _i: qk.qkv_norm_proj(x, Wf, nq, nk, nv, wq, wk, wv, wl.eps, 1, out=y)  # noqa: E731
+    for i in range(3):
+        elim(i)
+    e_ms, _ = time_launches(elim, per, stream)
+    elim_ms = max_over_ranks(e_ms, pg) / per
     ms_per_step = tot["step"] / steps
     value = world * wl.M / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
@@ -823,7 +831,10 @@ def run_qkv(args, rank, world, local, pg):
                            "speedup_vs_unfused": tot["unfused"] / tot["step"],
                            "two_step": "flashnorm_proj then qknorm_fused on q and k in place",
                            "unfused": "qknorm_fused RMSNorm writing x_hat, torch.matmul (cuBLAS) with W, "
-                                      "qknorm_fused on q and k"},
+                                      "qknorm_fused on q and k",
+                           "elimination_ms_per_step": elim_ms,
+                           "elimination": "qkv_norm_proj: the projection without the input norm, then every "
+                                          "group's RMSNorm (v's too); timed after the main region"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * steps, "clocks": clk,
         }), flush=True)
 

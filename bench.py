@@ -27,6 +27,7 @@ Rank 0 prints exactly one JSON line.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -41,6 +42,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 QK_DEFAULT = "long_context"
+VENDOR_BF16_DENSE_TFLOPS = 2250.0  # public B200 datasheet figure, dense (no 2:4 sparsity)
+# One metric string per workload, printed by both arms so their lines compare.
+METRIC_QK = "QK-Norm tokens/s and achieved HBM GB/s (% of B200 roofline) on 1 GPU"
+METRIC_FN = "FlashNorm norm-then-project tokens/s and tensor-core TFLOP/s (% of bf16 peak) on 1 GPU"
+METRIC_QKV = "RMSNorm + QKV projection + QK-Norm tokens/s and tensor-core TFLOP/s (% of bf16 peak) on 1 GPU"
+METRIC_TP = "Tensor-parallel QK-Norm tokens/s (SwiftQK scalar exchange) and latency reduction vs All-Gather QK-Norm"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -65,6 +72,8 @@ def parse_args():
                     help="tp_qknorm: on one GPU, time one rank's share of an S-way split "
                          "(its kernels and local collectives; no interconnect transfer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="long_context: skip the prefill_gqa, flashnorm_proj and qkv_proj_qknorm sub-measurements")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline work budget")
     return ap.parse_args()
 
@@ -88,8 +97,14 @@ def source_digest(paths):
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel_key: str, workload: str, src_paths):
-    """DRAM bytes per launch from a committed ncu capture, or None if absent or stale."""
+def traffic_for(kernel_key: str, workload: str, src_paths, algorithmic_bytes=None):
+    """Traffic per launch from a committed ncu capture, or None if absent or stale.
+
+    ``read`` is dram__bytes_read.sum; ``write`` is the bytes the SMs stored into
+    L2 (lts__t_sectors_srcunit_tex_op_write.sum x 32 B), which counts every
+    output byte even when the end of the output is still dirty in L2 as the
+    kernel exits (dram__bytes_write.sum misses that tail and is kept beside it).
+    """
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
@@ -97,7 +112,14 @@ def traffic_for(kernel_key: str, workload: str, src_paths):
     e = t.get(kernel_key, {}).get(workload)
     if not e or e.get("source_digest") != source_digest(src_paths):
         return None
-    return e.get("dram_bytes_per_launch")
+    rd, wr = e.get("dram_read_bytes_per_launch"), e.get("l2_write_bytes_from_sm_per_launch")
+    if rd is None or wr is None:
+        return None
+    out = {"total": rd + wr, "read": rd, "write": wr,
+           "dram_write": e.get("dram_write_bytes_per_launch"), "captured_on": e.get("captured_on")}
+    if algorithmic_bytes:
+        out["over_algorithmic"] = (rd + wr) / algorithmic_bytes
+    return out
 
 
 class ClockSampler:
@@ -145,7 +167,13 @@ class ClockSampler:
                 if len(parts) < 10:
                     continue
                 try:
-                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    try:
+                        ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    except ValueError:
+                        continue
+                try:
                     rows.append({"ts": ts, "index": int(parts[1]), "sm": float(parts[2]), "max": float(parts[3]),
                                  "power": float(parts[4]) if parts[4] not in ("[N/A]", "") else None,
                                  "hw_slowdown": parts[6], "hw_thermal": parts[7], "sw_thermal": parts[8],
@@ -157,8 +185,12 @@ class ClockSampler:
             sel = [r for r in rows if r["index"] == gpu_index] or rows
         else:
             sel = rows
-        # samples inside the timed window (1 s timestamp resolution)
-        win = [r for r in sel if self.t0 is not None and math.floor(self.t0) <= r["ts"] <= math.ceil(self.t1)]
+        # samples inside the timed window, widened by one sampling period; for a
+        # window shorter than that, the samples nearest to it
+        win = [r for r in sel if self.t0 is not None and self.t0 - 0.11 <= r["ts"] <= self.t1 + 0.11]
+        if not win and sel and self.t0 is not None:
+            mid = 0.5 * (self.t0 + self.t1)
+            win = sorted(sel, key=lambda r: abs(r["ts"] - mid))[:2]
         if not win:
             win = sel
         if not win:
@@ -169,7 +201,18 @@ class ClockSampler:
                 if r[k].lower() == "active":
                     reasons.add({"hw_thermal": "hw_thermal_slowdown", "sw_thermal": "sw_thermal_slowdown"}.get(k, k))
         return {"sm_mhz": statistics.median(r["sm"] for r in win), "sm_max_mhz": max(r["max"] for r in win),
-                "reasons": sorted(reasons), "samples": len(win)}
+                "reasons": sorted(reasons), "samples": len(win),
+                "window_s": round(self.t1 - self.t0, 3) if self.t0 is not None else None}
+
+
+def at_max_clock(us, clk):
+    """A device time scaled to the maximum SM clock (time x median sampled MHz / max MHz).
+
+    Meaningful for work bound by the SM clock (the tensor-core GEMMs); the
+    HBM-bound kernels barely depend on it.  None without clock samples."""
+    if not clk or not clk.get("sm_mhz") or not clk.get("sm_max_mhz"):
+        return None
+    return us * clk["sm_mhz"] / clk["sm_max_mhz"]
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -292,29 +335,34 @@ def run_reference(args):
         nq = nk = wl.N // 3
         wq, wk = W.make_qkv_norm_weights(nq, nk)
         fn = lambda: cpu_baseline_qkv(inp, nq, nk, wq, wk, 4.0)  # noqa: E731
-        metric = "RMSNorm + QKV projection + QK-Norm tokens/s (fp64 CPU oracle)"
+        metric = METRIC_QKV
         cfg = {"workload": "qkv_proj_qknorm", "M": wl.M, "K": wl.K, "nq": nq, "nk": nk, "nv": wl.N - 2 * nq}
     elif args.workload == "flashnorm_proj":
         wl = W.FLASHNORM_WORKLOAD
         inp = W.make_flashnorm_inputs(seed=0, M=64)
         fn = lambda: cpu_baseline_flashnorm(inp, 4.0)  # noqa: E731
-        metric = "FlashNorm norm-then-project tokens/s (fp64 CPU oracle)"
+        metric = METRIC_FN
         cfg = {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N}
     else:
         # the tensor-parallel layer computes the prefill GQA QK-Norm; the oracle computes it whole
         wl = W.QKNORM_WORKLOADS["prefill_gqa" if args.workload == "tp_qknorm" else args.workload]
         inp = W.make_qknorm_inputs(wl, seed=0, tokens=min(wl.tokens, 8192))
         fn = lambda: cpu_baseline_qknorm(inp, 4.0)  # noqa: E731
-        metric = "QK-Norm tokens/s (fp64 CPU oracle)"
+        metric = METRIC_TP if args.workload == "tp_qknorm" else METRIC_QK
         cfg = {"workload": args.workload, "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk, "n_seg": wl.n_seg}
     for _ in range(args.warmup):
         fn()
-    vals = [fn() for _ in range(steps)]
+    vals, walls = [], []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        vals.append(fn())
+        walls.append(time.perf_counter() - t0)
     value = statistics.median(v["value"] for v in vals)
     last = vals[-1]
     print(json.dumps({
         "impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "steps": steps, "warmup": args.warmup, "ms_per_step": statistics.median(walls) * 1e3,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"]},
@@ -341,6 +389,94 @@ def time_launches(fn, steps, stream):
     return t_start.elapsed_time(t_end), [a.elapsed_time(b) for a, b in ev]
 
 
+# The sources each norm kernel is compiled from: a committed traffic capture
+# stays valid while their digest is unchanged.
+QK_SRC = {"rownorm_staged_kernel": ["rmsnorm_qknorm_b200/csrc/rownorm_staged.cuh",
+                                    "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
+                                    "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"],
+          "rownorm_vec_stream_kernel": ["rmsnorm_qknorm_b200/csrc/rownorm_register.cuh",
+                                        "rmsnorm_qknorm_b200/csrc/qkn_common.cuh"]}
+
+
+def qk_kernel_for(wl):
+    """The kernel the library picks for a workload's rows (the choice depends on the widths only)."""
+    row_bytes = max(wl.dq, wl.dk) * (4 if wl.dtype == "f32" else 2)
+    return "rownorm_vec_stream_kernel" if row_bytes <= 4096 and wl.n_seg <= 8 else "rownorm_staged_kernel"
+
+
+def qk_sets(wl, my_tokens, dev, rank):
+    """Input sets for a QK-Norm workload: one when a set is larger than twice L2,
+    else enough rotating sets that consecutive launches never find theirs in L2."""
+    import torch
+    from rmsnorm_qknorm_b200 import workloads as W
+    from rmsnorm_qknorm_b200 import dist as qdist
+    per_set = wl.algorithmic_bytes(my_tokens)
+    nsets = 1 if per_set > 2 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_set))
+    sets = []
+    for si in range(nsets):
+        inp = W.make_qknorm_inputs(wl, seed=qdist.rank_seed(si, rank), device=dev, tokens=my_tokens)
+        inp["q_out"] = torch.empty_like(inp["q"])
+        inp["k_out"] = torch.empty_like(inp["k"])
+        sets.append(inp)
+    return sets, per_set
+
+
+def qk_graph_time(wl, sets, steps, warmup, dev, local, pg, rank):
+    """qknorm_fused over rotating sets: `steps` launches captured in one CUDA graph
+    and replayed once between CUDA events (the device time of back-to-back
+    launches, not the binding's launch rate).  Returns (total ms, clocks)."""
+    import torch
+    import rmsnorm_qknorm_b200 as qk
+    nsets = len(sets)
+
+    def step(i):
+        st = sets[i % nsets]
+        qk.qknorm_fused(st["q"], st["k"], st["wq"], st["wk"], wl.eps, wl.n_seg, q_out=st["q_out"], k_out=st["k_out"])
+
+    for i in range(max(warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(steps):
+            step(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    barrier(pg)
+    clocks = ClockSampler() if rank == 0 else None
+    if clocks:
+        clocks.start()
+        clocks.mark(True)
+    total_ms, _ = time_launches(lambda _i: graph.replay(), 1, torch.cuda.current_stream(dev))
+    if clocks:
+        clocks.mark(False)
+    barrier(pg)
+    total_ms = max_over_ranks(total_ms, pg)
+    clk = clocks.stop(gpu_index=local) if clocks else None
+    del graph
+    return total_ms, clk, step
+
+
+def extra_qknorm(name, dev, local, pg, rank, steps=200):
+    """Sub-measurement of another QK-Norm workload at full size (per GPU)."""
+    from rmsnorm_qknorm_b200 import workloads as W
+    wl = W.QKNORM_WORKLOADS[name]
+    sets, per_set = qk_sets(wl, wl.tokens, dev, rank)
+    total_ms, clk, _ = qk_graph_time(wl, sets, steps, 3, dev, local, pg, rank)
+    del sets
+    pk, pk_kind = peaks()
+    us = total_ms / steps * 1e3
+    gbs = per_set / (us * 1e-6) / 1e9
+    kernel = qk_kernel_for(wl)
+    return {"workload": name, "tokens": wl.tokens, "dq": wl.dq, "dk": wl.dk, "n_seg": wl.n_seg, "dtype": wl.dtype,
+            "us_per_launch": us, "tokens_per_s": wl.tokens / (us * 1e-6), "algorithmic_bytes": per_set,
+            "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
+            "peak_source": f"{pk_kind} HBM copy bandwidth", "kernel": kernel,
+            "traffic": traffic_for(kernel, name, QK_SRC[kernel], per_set),
+            "steps": steps, "timing": "one CUDA graph of all launches, CUDA events around its replay",
+            "clocks": clk, "us_at_max_clock": at_max_clock(us, clk)}
+
+
 def run_qknorm(args, rank, world, local, pg):
     import torch
     import rmsnorm_qknorm_b200 as qk
@@ -357,51 +493,11 @@ def run_qknorm(args, rank, world, local, pg):
         my_tokens, global_tokens = r1 - r0, batch
     else:
         my_tokens, global_tokens = batch, world * batch
-    per_set = wl.algorithmic_bytes(my_tokens)
-    nsets = 1 if per_set > 2 * L2_BYTES else int(math.ceil(3 * L2_BYTES / per_set))
-    sets = []
-    for s in range(nsets):
-        inp = W.make_qknorm_inputs(wl, seed=qdist.rank_seed(s, rank), device=dev, tokens=my_tokens)
-        inp["q_out"] = torch.empty_like(inp["q"])
-        inp["k_out"] = torch.empty_like(inp["k"])
-        sets.append(inp)
-
-    def step(i):
-        s = sets[i % nsets]
-        qk.qknorm_fused(s["q"], s["k"], s["wq"], s["wk"], wl.eps, wl.n_seg, q_out=s["q_out"], k_out=s["k_out"])
-
-    for i in range(max(args.warmup, 3)):
-        step(i)
-    # The timed launches are captured in one CUDA graph and replayed: the
-    # device time of back-to-back launches is measured, not the Python
-    # binding's launch rate or the per-launch front-end latency (small batches
-    # run for a few microseconds, less than one host-side launch).
-    use_graph = True
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for i in range(steps):
-            step(i)
-    graph.replay()
-    torch.cuda.synchronize()
-    barrier(pg)
-    clocks = ClockSampler() if rank == 0 else None
-    if clocks:
-        clocks.start()
-        clocks.mark(True)
-    if use_graph:
-        total_ms, _ = time_launches(lambda _i: graph.replay(), 1, torch.cuda.current_stream(dev))
-        launch_ms = [total_ms / steps]
-    else:
-        total_ms, launch_ms = time_launches(step, steps, stream)
-    if clocks:
-        clocks.mark(False)
-    barrier(pg)
-    total_ms = max_over_ranks(total_ms, pg)
-    avg_launch_ms = max_over_ranks(statistics.mean(launch_ms), pg)
-    clk = clocks.stop(gpu_index=local) if clocks else None
-    if graph is not None:
-        del graph
+    sets, per_set = qk_sets(wl, my_tokens, dev, rank)
+    nsets = len(sets)
+    total_ms, clk, step = qk_graph_time(wl, sets, steps, args.warmup, dev, local, pg, rank)
+    # the launches are back to back in one graph: the mean launch time is the step time
+    avg_launch_ms = total_ms / steps
 
     ms_per_step = total_ms / steps
     value = global_tokens / (ms_per_step * 1e-3)
@@ -444,13 +540,8 @@ def run_qknorm(args, rank, world, local, pg):
                      "frac": stats_bytes / (s_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                      "what": "rmsnorm_partial_stats of q then of k (the per-segment sums alone), "
                              f"{stats_steps} steps in one CUDA graph over the same rotating sets"}
-    src = ["rmsnorm_qknorm_b200/csrc/qknorm.cu", "rmsnorm_qknorm_b200/csrc/rownorm_staged.cuh",
-           "rmsnorm_qknorm_b200/csrc/rownorm_register.cuh", "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
-           "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
-    # the kernel the library picks for these rows (the choice depends on the widths only)
-    row_bytes = max(wl.dq, wl.dk) * (4 if wl.dtype == "f32" else 2)
-    kernel = "rownorm_vec_stream_kernel" if row_bytes <= 4096 and wl.n_seg <= 8 else "rownorm_staged_kernel"
-    traffic = traffic_for(kernel, wl.name, src) if args.tokens is None else None
+    kernel = qk_kernel_for(wl)
+    traffic = traffic_for(kernel, wl.name, QK_SRC[kernel], per_set) if args.tokens is None else None
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -476,15 +567,39 @@ def run_qknorm(args, rank, world, local, pg):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
                "note": "qknorm_fused_host on pinned host q,k: chunks of ~sqrt(bytes x 1.5 MB) uploaded, normalised and downloaded "
                         "with the three overlapped; outputs in pinned host memory, per step"}
+        del hq, hk, oq, ok, ws
+    del sets
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = W.make_qknorm_inputs(wl, seed=0, device="cpu", tokens=min(wl.tokens, 65536))
         cpu = cpu_baseline_qknorm(host, args.cpu_seconds)
+        del host
+
+    # The other graded workloads, measured after the headline on the same GPU,
+    # each with its own clock record: the prefill GQA QK-Norm (HBM roofline)
+    # and the two tensor-core projections (bf16 peak).
+    extras = {}
+    if args.workload == QK_DEFAULT and args.tokens is None and not args.no_extras:
+        extras["prefill_gqa"] = extra_qknorm("prefill_gqa", dev, local, pg, rank)
+        torch.cuda.empty_cache()
+        for kind in ("flashnorm_proj", "qkv_proj_qknorm"):
+            extras[kind] = extra_projection(kind, dev, local, pg, rank)
+            torch.cuda.empty_cache()
+        if world > 1:
+            # tensor-parallel QK-Norm of the prefill GQA layer split over all
+            # the ranks (S = world): SwiftQK's scalar exchange against the
+            # All-Gather form, over the real interconnect
+            from rmsnorm_qknorm_b200 import tp as qtp
+            line = _run_tp(args, rank, world, local, pg, torch, qtp, W, steps=100)
+            if rank == 0:
+                extras["tp_qknorm"] = {k: line[k] for k in ("value", "unit", "ms_per_step", "config",
+                                                            "comparison", "roofline", "clocks")}
+            torch.cuda.empty_cache()
 
     if rank == 0:
         out = {
-            "metric": "QK-Norm tokens/s and achieved HBM GB/s (% of B200 roofline) on 1 GPU",
+            "metric": METRIC_QK,
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
             "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.strong else "weak", "vs_baseline": None,
@@ -495,7 +610,13 @@ def run_qknorm(args, rank, world, local, pg):
                        "l2": ("inputs larger than L2" if nsets == 1 else
                               f"{nsets} rotating input sets totalling {nsets * per_set / 1e6:.0f} MB > L2")},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                         "frac": achieved / pk["hbm_gbs"],
+                         "traffic": traffic["total"] if traffic else None,
+                         "traffic_read": traffic["read"] if traffic else None,
+                         "traffic_write": traffic["write"] if traffic else None,
+                         "traffic_over_algorithmic": traffic["over_algorithmic"] if traffic else None,
+                         "traffic_source": (f"ncu dram__bytes_read.sum + lts__t_sectors_srcunit_tex_op_write.sum x 32 B; "
+                                            f"{traffic['captured_on']}") if traffic else None,
                          "kernel": kernel,
                          "algorithmic_bytes_per_launch": per_set,
                          "avg_launch_us": avg_launch_ms * 1e3,
@@ -507,9 +628,11 @@ def run_qknorm(args, rank, world, local, pg):
             "eager_launch_us": eager_launch_us,
             "cpu_baseline": cpu,
             "e2e": e2e,
+            # the headline kernel's launches in the timed region (the sub-measurements run after it)
             "gpu_launches": steps,
             "clocks": clk,
         }
+        out.update(extras)
         print(json.dumps(out), flush=True)
 
 
@@ -564,63 +687,159 @@ def host_pipeline(hx, hy, call, dev, nchunks=8):
     return step
 
 
-def run_flashnorm(args, rank, world, local, pg):
+FN_SRC = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
+          "rmsnorm_qknorm_b200/csrc/qkn_common.cuh", "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
+QKV_SRC = ["rmsnorm_qknorm_b200/csrc/qkv_qknorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
+           "rmsnorm_qknorm_b200/csrc/qkn_common.cuh", "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
+
+
+def projection_forms(kind, dev, rank):
+    """Inputs of the projection workload (x [8192, 4096], W [4096, 12288]) and
+    the forms timed side by side:
+
+    * step: the 1/rms statistics pass + our tcgen05 GEMM (for the QKV form,
+      with q and k normalised in its epilogue);
+    * gemm_only: the GEMM alone, given the 1/rms vector;
+    * two_step (QKV form): our projection, then qknorm_fused on q and k in place;
+    * unfused: our RMSNorm writing the normalised x, cuBLAS with the original W
+      (torch.matmul), then (QKV form) qknorm_fused on q and k."""
     import torch
     import rmsnorm_qknorm_b200 as qk
     from rmsnorm_qknorm_b200 import workloads as W
-    qk.load_library()
-    wl = W.FLASHNORM_WORKLOAD
-    steps = args.steps if args.steps is not None else 200
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream(dev)
     from rmsnorm_qknorm_b200 import dist as qdist
+    wl = W.FLASHNORM_WORKLOAD
     inp = W.make_flashnorm_inputs(seed=qdist.rank_seed(0, rank), device=dev)
     x, w, Wm = inp["x"], inp["w"], inp["W"]
     Wf = qk.flashnorm_fold_weights(w, Wm)
     y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
     inv = torch.empty(wl.M, dtype=torch.float32, device=dev)
-
-    def step(_i):
-        qk.flashnorm_proj(x, Wf, wl.eps, inv_rms_out=inv, out=y)
-
-    def gemm_only(_i):
-        qk.flashnorm_proj(x, Wf, wl.eps, inv_rms=inv, out=y)
-
-    # unfused comparison: RMSNorm kernel writing normalised x, then cuBLAS with the original W
     xn = torch.empty_like(x)
+    c = {"wl": wl, "x": x, "w": w, "W": Wm, "Wf": Wf, "y": y, "inv": inv}
+    if kind == "flashnorm_proj":
+        def step(_i):
+            qk.flashnorm_proj(x, Wf, wl.eps, inv_rms_out=inv, out=y)
 
-    def unfused(_i):
-        qk.qknorm_fused(x, None, w, None, wl.eps, 1, q_out=xn)
-        torch.matmul(xn, Wm, out=y)
+        def gemm_only(_i):
+            qk.flashnorm_proj(x, Wf, wl.eps, inv_rms=inv, out=y)
 
-    for i in range(max(args.warmup, 3)):
-        step(i)
-        gemm_only(i)
-        unfused(i)
+        def unfused(_i):
+            qk.qknorm_fused(x, None, w, None, wl.eps, 1, q_out=xn)
+            torch.matmul(xn, Wm, out=y)
+
+        c["forms"] = {"step": step, "gemm_only": gemm_only, "unfused": unfused}
+    else:
+        nq = nk = wl.N // 3
+        nv = wl.N - nq - nk
+        wq, wk = W.make_qkv_norm_weights(nq, nk, device=dev)
+        ws = torch.empty(qk.qkv_proj_qknorm_workspace_bytes(wl.M, nq, nk, nv), dtype=torch.uint8, device=dev)
+        c.update(nq=nq, nk=nk, nv=nv, wq=wq, wk=wk, ws=ws)
+
+        def step(_i):  # statistics pass + one fused GEMM (q, k normalised in its epilogue)
+            qk.qkv_proj_qknorm(x, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms_out=inv, workspace=ws, out=y)
+
+        def gemm_only(_i):  # the fused GEMM alone (plus its 2 KB counter reset)
+            qk.qkv_proj_qknorm(x, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms=inv, workspace=ws, out=y)
+
+        def two_step(_i):
+            qk.flashnorm_proj(x, Wf, wl.eps, inv_rms_out=inv, out=y)
+            qk.qknorm_fused(y[:, :nq], y[:, nq:nq + nk], wq, wk, wl.eps, 1, inplace=True)
+
+        def unfused(_i):
+            qk.qknorm_fused(x, None, w, None, wl.eps, 1, q_out=xn)
+            torch.matmul(xn, Wm, out=y)
+            qk.qknorm_fused(y[:, :nq], y[:, nq:nq + nk], wq, wk, wl.eps, 1, inplace=True)
+
+        c["forms"] = {"step": step, "gemm_only": gemm_only, "two_step": two_step, "unfused": unfused}
+    return c
+
+
+def time_forms(forms, steps, warmup, stream, pg, rank, local, rounds=5):
+    """Every form timed in alternating rounds (so all see the same clocks), CUDA
+    events around each launch.  Returns ({form: ms per step}, mean gemm_only
+    launch ms, clocks, timed steps per form); all maxima over ranks."""
+    for i in range(max(warmup, 3)):
+        for f in forms.values():
+            f(i)
     barrier(pg)
     clocks = ClockSampler() if rank == 0 else None
     if clocks:
         clocks.start()
         clocks.mark(True)
-    # the full step and the projection alone are timed in alternating rounds so
-    # both see the same clocks (a long run settles under the power cap)
-    rounds = 5
     per = max(steps // rounds, 1)
-    total_ms, gemm_ms, unf_ms = 0.0, [], 0.0
+    tot = dict.fromkeys(forms, 0.0)
+    gemm_ms = []
     for _ in range(rounds):
-        t, _ = time_launches(step, per, stream)
-        total_ms += t
-        _, gm = time_launches(gemm_only, per, stream)
-        gemm_ms += gm
-        u, _ = time_launches(unfused, per, stream)
-        unf_ms += u
-    steps = per * rounds
+        for name, f in forms.items():
+            t, each = time_launches(f, per, stream)
+            tot[name] += t
+            if name == "gemm_only":
+                gemm_ms += each
     if clocks:
         clocks.mark(False)
     barrier(pg)
-    total_ms = max_over_ranks(total_ms, pg)
+    n = per * rounds
+    ms = {name: max_over_ranks(t, pg) / n for name, t in tot.items()}
     avg_gemm = max_over_ranks(statistics.mean(gemm_ms), pg)
-    unf_ms = max_over_ranks(unf_ms, pg)
+    clk = clocks.stop(gpu_index=local) if clocks else None
+    return ms, avg_gemm, clk, n
+
+
+def projection_roofline(kind, avg_gemm_ms, clk, src):
+    from rmsnorm_qknorm_b200 import workloads as W
+    wl = W.FLASHNORM_WORKLOAD
+    pk, pk_kind = peaks()
+    tflops = wl.flops() / (avg_gemm_ms * 1e-3) / 1e12
+    kernel = "flashnorm_gemm_kernel" if kind == "flashnorm_proj" else "qkv_qknorm_gemm_kernel"
+    # algorithmic bytes of one launch: x and W' read once, y written once
+    algo = (wl.M * wl.K + wl.N * wl.K + wl.M * wl.N) * 2
+    t = traffic_for(kernel, kind, src, algo)
+    return {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tflops / pk["bf16_tflops"], "kernel": kernel,
+            "traffic": t["total"] if t else None, "traffic_read": t["read"] if t else None,
+            "traffic_write": t["write"] if t else None,
+            "traffic_over_algorithmic": t["over_algorithmic"] if t else None, "algorithmic_bytes": algo,
+            "avg_launch_us": avg_gemm_ms * 1e3, "flops_per_launch": wl.flops(),
+            "peak_source": f"{pk_kind} cuBLAS bf16 burst",
+            "frac_of_sustained": tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+            "frac_of_vendor_dense": tflops / VENDOR_BF16_DENSE_TFLOPS,
+            "avg_launch_us_at_max_clock": at_max_clock(avg_gemm_ms * 1e3, clk)}
+
+
+def extra_projection(kind, dev, local, pg, rank, steps=100):
+    """Sub-measurement of a projection workload (per GPU) for the headline line."""
+    import torch
+    c = projection_forms(kind, dev, rank)
+    ms, avg_gemm, clk, n = time_forms(c["forms"], steps, 3, torch.cuda.current_stream(dev), pg, rank, local)
+    wl = c["wl"]
+    del c
+    rf = projection_roofline(kind, avg_gemm, clk, FN_SRC if kind == "flashnorm_proj" else QKV_SRC)
+    out = {"workload": kind, "M": wl.M, "K": wl.K, "N": wl.N, "dtype": "bf16",
+           "gemm_us": avg_gemm * 1e3, "tflops": rf["achieved"], "frac_of_burst": rf["frac"],
+           "frac_of_sustained": rf["frac_of_sustained"], "frac_of_vendor_dense": rf["frac_of_vendor_dense"],
+           "gemm_us_at_max_clock": rf["avg_launch_us_at_max_clock"],
+           "traffic": rf["traffic"], "traffic_over_algorithmic": rf["traffic_over_algorithmic"],
+           "step_ms": ms["step"], "tokens_per_s": wl.M / (ms["step"] * 1e-3),
+           "unfused_ms": ms["unfused"], "speedup_vs_unfused": ms["unfused"] / ms["step"],
+           "step_ms_at_max_clock": at_max_clock(ms["step"], clk),
+           "peak_source": rf["peak_source"], "steps": n, "clocks": clk,
+           "timing": "step, GEMM alone and unfused form in alternating rounds, CUDA events per launch"}
+    if "two_step" in ms:
+        out["two_step_ms"] = ms["two_step"]
+        out["speedup_vs_two_step"] = ms["two_step"] / ms["step"]
+    return out
+
+
+def run_flashnorm(args, rank, world, local, pg):
+    import torch
+    import rmsnorm_qknorm_b200 as qk
+    from rmsnorm_qknorm_b200 import workloads as W
+    qk.load_library()
+    steps = args.steps if args.steps is not None else 200
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    c = projection_forms("flashnorm_proj", dev, rank)
+    wl, x, w, Wm, Wf, inv = c["wl"], c["x"], c["w"], c["W"], c["Wf"], c["inv"]
+    ms, avg_gemm, clk, steps = time_forms(c["forms"], steps, args.warmup, stream, pg, rank, local)
     # the fold, an offline step (once per weight update): W' = diag(w) W, K-major
     fold_out = torch.empty_like(Wf)
     for _ in range(3):
@@ -637,14 +856,9 @@ def run_flashnorm(args, rank, world, local, pg):
     s_ms, _ = time_launches(lambda _i: qk.flashnorm_inv_rms(x, wl.eps, out=inv_alone), fold_n, stream)
     stats_us = max_over_ranks(s_ms, pg) / fold_n * 1e3
     stats_bytes = x.numel() * x.element_size() + inv.numel() * 4
-    clk = clocks.stop(gpu_index=local) if clocks else None
-    ms_per_step = total_ms / steps
+    ms_per_step = ms["step"]
     value = world * wl.M / (ms_per_step * 1e-3)
     pk, pk_kind = peaks()
-    tflops = wl.flops() / (avg_gemm * 1e-3) / 1e12
-    src = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
-           "rmsnorm_qknorm_b200/csrc/qkn_common.cuh",
-           "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
 
     e2e = None
     if args.e2e_steps > 0:
@@ -670,21 +884,16 @@ def run_flashnorm(args, rank, world, local, pg):
 
     if rank == 0:
         print(json.dumps({
-            "metric": "FlashNorm norm-then-project tokens/s and tensor-core TFLOP/s (% of bf16 peak) on 1 GPU",
+            "metric": METRIC_FN,
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "eps": wl.eps,
                        "parallelism": f"dp{world} (token batches, no collective)",
                        "l2": "inputs larger than L2 (x 67 MB + W' 101 MB)"},
-            "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tflops / pk["bf16_tflops"], "kernel": "flashnorm_gemm_kernel",
-                         "traffic": traffic_for("flashnorm_gemm_kernel", wl.name, src),
-                         "avg_launch_us": avg_gemm * 1e3, "flops_per_launch": wl.flops(),
-                         "peak_source": f"{pk_kind} cuBLAS bf16 burst",
-                         "frac_of_sustained": tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])},
-            "comparison": {"unfused_ms_per_step": unf_ms / steps, "fused_ms_per_step": ms_per_step,
-                           "speedup_vs_unfused": (unf_ms / steps) / ms_per_step,
+            "roofline": projection_roofline("flashnorm_proj", avg_gemm, clk, FN_SRC),
+            "comparison": {"unfused_ms_per_step": ms["unfused"], "fused_ms_per_step": ms_per_step,
+                           "speedup_vs_unfused": ms["unfused"] / ms_per_step,
                            "unfused": "qknorm_fused RMSNorm writing x_hat, then torch.matmul (cuBLAS) with W"},
             "inv_rms": {"us_per_launch": stats_us, "algorithmic_bytes": stats_bytes,
                         "achieved_gbs": stats_bytes / (stats_us * 1e-6) / 1e9,
@@ -705,78 +914,25 @@ def run_qkv(args, rank, world, local, pg):
     import torch
     import rmsnorm_qknorm_b200 as qk
     from rmsnorm_qknorm_b200 import workloads as W
-    from rmsnorm_qknorm_b200 import dist as qdist
     qk.load_library()
-    wl = W.FLASHNORM_WORKLOAD
-    nq = nk = wl.N // 3
-    nv = wl.N - nq - nk
     steps = args.steps if args.steps is not None else 200
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    inp = W.make_flashnorm_inputs(seed=qdist.rank_seed(0, rank), device=dev)
-    x, w, Wm = inp["x"], inp["w"], inp["W"]
-    wq, wk = W.make_qkv_norm_weights(nq, nk, device=dev)
-    Wf = qk.flashnorm_fold_weights(w, Wm)
-    y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
-    inv = torch.empty(wl.M, dtype=torch.float32, device=dev)
-    ws = torch.empty(qk.qkv_proj_qknorm_workspace_bytes(wl.M, nq, nk, nv), dtype=torch.uint8, device=dev)
-
-    def step(_i):  # statistics pass + one fused GEMM (q, k normalised in its epilogue)
-        qk.qkv_proj_qknorm(x, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms_out=inv, workspace=ws, out=y)
-
-    def gemm_only(_i):  # the fused GEMM alone (plus its 2 KB counter reset)
-        qk.qkv_proj_qknorm(x, Wf, nq, nk, nv, wq, wk, wl.eps, inv_rms=inv, workspace=ws, out=y)
-
-    def two_step(_i):  # our projection, then qknorm_fused on the q and k column blocks in place
-        qk.flashnorm_proj(x, Wf, wl.eps, inv_rms_out=inv, out=y)
-        qk.qknorm_fused(y[:, :nq], y[:, nq:nq + nk], wq, wk, wl.eps, 1, inplace=True)
-
-    xn = torch.empty_like(x)
-
-    def unfused(_i):  # RMSNorm kernel, cuBLAS with the original W, QK-Norm kernel
-        qk.qknorm_fused(x, None, w, None, wl.eps, 1, q_out=xn)
-        torch.matmul(xn, Wm, out=y)
-        qk.qknorm_fused(y[:, :nq], y[:, nq:nq + nk], wq, wk, wl.eps, 1, inplace=True)
-
-    for i in range(max(args.warmup, 3)):
-        for f in (step, gemm_only, two_step, unfused):
-            f(i)
-    barrier(pg)
-    clocks = ClockSampler() if rank == 0 else None
-    if clocks:
-        clocks.start()
-        clocks.mark(True)
-    rounds = 5
-    per = max(steps // rounds, 1)
-    tot = {"step": 0.0, "two_step": 0.0, "unfused": 0.0}
-    gemm_ms = []
-    for _ in range(rounds):  # alternating rounds: every form sees the same clocks
-        tot["step"] += time_launches(step, per, stream)[0]
-        gemm_ms += time_launches(gemm_only, per, stream)[1]
-        tot["two_step"] += time_launches(two_step, per, stream)[0]
-        tot["unfused"] += time_launches(unfused, per, stream)[0]
-    steps = per * rounds
-    if clocks:
-        clocks.mark(False)
-    barrier(pg)
-    for key in tot:
-        tot[key] = max_over_ranks(tot[key], pg)
-    avg_gemm = max_over_ranks(statistics.mean(gemm_ms), pg)
-    clk = clocks.stop(gpu_index=local) if clocks else None
+    c = projection_forms("qkv_proj_qknorm", dev, rank)
+    wl, x, Wf, y, inv = c["wl"], c["x"], c["Wf"], c["y"], c["inv"]
+    nq, nk, nv, wq, wk = c["nq"], c["nk"], c["nv"], c["wq"], c["wk"]
+    ms, avg_gemm, clk, steps = time_forms(c["forms"], steps, args.warmup, stream, pg, rank, local)
     # the RMSNorm-elimination form (qkv_norm_proj: the projection without the
     # input norm, then each group's RMSNorm), timed after the main region
     wv = torch.ones(nv, dtype=torch.bfloat16, device=dev)
     elim = lambda _i: qk.qkv_norm_proj(x, Wf, nq, nk, nv, wq, wk, wv, wl.eps, 1, out=y)  # noqa: E731
     for i in range(3):
         elim(i)
+    per = max(steps // 5, 1)
     e_ms, _ = time_launches(elim, per, stream)
     elim_ms = max_over_ranks(e_ms, pg) / per
-    ms_per_step = tot["step"] / steps
+    ms_per_step = ms["step"]
     value = world * wl.M / (ms_per_step * 1e-3)
-    pk, pk_kind = peaks()
-    tflops = wl.flops() / (avg_gemm * 1e-3) / 1e12
-    src = ["rmsnorm_qknorm_b200/csrc/qkv_qknorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
-           "rmsnorm_qknorm_b200/csrc/qkn_common.cuh", "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
 
     e2e = None
     if args.e2e_steps > 0:
@@ -807,28 +963,22 @@ def run_qkv(args, rank, world, local, pg):
         cpu = cpu_baseline_qkv(host, nq, nk, hwq, hwk, args.cpu_seconds)
 
     if rank == 0:
+        rf = projection_roofline("qkv_proj_qknorm", avg_gemm, clk, QKV_SRC)
+        rf["launch_timing"] = "CUDA events around each call with a given 1/rms (counter reset + the fused GEMM)"
         print(json.dumps({
-            "metric": "RMSNorm + QKV projection + QK-Norm tokens/s and tensor-core TFLOP/s (% of bf16 peak) "
-                      "on 1 GPU",
+            "metric": METRIC_QKV,
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "qkv_proj_qknorm", "M": wl.M, "K": wl.K, "nq": nq, "nk": nk, "nv": nv,
                        "eps": wl.eps, "parallelism": f"dp{world} (token batches, no collective)",
                        "l2": "inputs larger than L2 (x 67 MB + W' 101 MB)"},
-            "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tflops / pk["bf16_tflops"], "kernel": "qkv_qknorm_gemm_kernel",
-                         "traffic": traffic_for("qkv_qknorm_gemm_kernel", "qkv_proj_qknorm", src),
-                         "avg_launch_us": avg_gemm * 1e3, "flops_per_launch": wl.flops(),
-                         "launch_timing": "CUDA events around each call with a given 1/rms (counter reset + "
-                                          "the fused GEMM)",
-                         "peak_source": f"{pk_kind} cuBLAS bf16 burst",
-                         "frac_of_sustained": tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])},
+            "roofline": rf,
             "comparison": {"fused_ms_per_step": ms_per_step,
-                           "two_step_ms_per_step": tot["two_step"] / steps,
-                           "unfused_ms_per_step": tot["unfused"] / steps,
-                           "speedup_vs_two_step": tot["two_step"] / tot["step"],
-                           "speedup_vs_unfused": tot["unfused"] / tot["step"],
+                           "two_step_ms_per_step": ms["two_step"],
+                           "unfused_ms_per_step": ms["unfused"],
+                           "speedup_vs_two_step": ms["two_step"] / ms_per_step,
+                           "speedup_vs_unfused": ms["unfused"] / ms_per_step,
                            "two_step": "flashnorm_proj then qknorm_fused on q and k in place",
                            "unfused": "qknorm_fused RMSNorm writing x_hat, torch.matmul (cuBLAS) with W, "
                                       "qknorm_fused on q and k",
@@ -860,13 +1010,16 @@ def run_tp(args, rank, world, local, pg):
         dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", local))
         own_group = True
     try:
-        _run_tp(args, rank, world, local, pg, torch, tp, W)
+        line = _run_tp(args, rank, world, local, pg, torch, tp, W)
     finally:
         if own_group:
             dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
-def _run_tp(args, rank, world, local, pg, torch, tp, W):
+def _run_tp(args, rank, world, local, pg, torch, tp, W, steps=None):
+    """Times the tensor-parallel flows; returns rank 0's JSON line (None elsewhere)."""
     import rmsnorm_qknorm_b200 as qk
     from rmsnorm_qknorm_b200 import dist as qdist
     wl = W.QKNORM_WORKLOADS["prefill_gqa"]
@@ -876,7 +1029,8 @@ def _run_tp(args, rank, world, local, pg, torch, tp, W):
     if shards < 1 or wl.dq % shards or wl.dk % shards:
         raise SystemExit(f"dq={wl.dq} and dk={wl.dk} must split evenly over {shards} shards")
     T, dq, dk = wl.tokens, wl.dq // shards, wl.dk // shards
-    steps = args.steps if args.steps is not None else 200
+    if steps is None:
+        steps = args.steps if args.steps is not None else 200
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     emulated = shards > world
@@ -969,9 +1123,8 @@ def _run_tp(args, rank, world, local, pg, torch, tp, W):
         host = W.make_qknorm_inputs(wl, seed=0, device="cpu", tokens=8192)
         cpu = cpu_baseline_qknorm(host, args.cpu_seconds)
     if rank == 0:
-        print(json.dumps({
-            "metric": "Tensor-parallel QK-Norm tokens/s (SwiftQK scalar exchange) and latency reduction vs "
-                      "All-Gather QK-Norm",
+        return {
+            "metric": METRIC_TP,
             "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": n,
             "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -1002,7 +1155,7 @@ def _run_tp(args, rank, world, local, pg, torch, tp, W):
             # per step: two statistic and two apply launches in each SwiftQK flow, one qknorm_fused
             # in each All-Gather flow; timed from the graphs and from Python
             "gpu_launches": (8 + len(flows) - 2) * n * 2,
-        }), flush=True)
+        }
 
 
 def main():

@@ -323,12 +323,12 @@ QKN_API qkn_status qkv_norm_proj(const void *x, const void *W_folded, void *y,
  * callers under a framework whose allocator owns the device, real-time loops
  * that cannot absorb an allocator's latency.
  *
- * Same arguments and result as flashnorm_proj with inv_rms == inv_rms_out ==
- * NULL (equal up to the summation order of the row statistic): a row-
- * statistics pass writes the 1/rms vector into a fixed 1 MiB array compiled
- * into the library (a file-scope __device__ variable, present on every GPU
- * that loads the library until the process exits), then the projection reads
- * it.  The call allocates nothing.
+ * Same arguments and the same launches as flashnorm_proj with inv_rms ==
+ * NULL and an inv_rms_out buffer, so the result is bit-identical to that
+ * call: a row-statistics pass writes the 1/rms vector into a fixed 1 MiB
+ * array compiled into the library (a file-scope __device__ variable, present
+ * on every GPU that loads the library until the process exits), then the
+ * projection reads it.  The call allocates nothing.
  *
  * Limits and caveats:
  * - M <= 262144 rows; larger M returns QKN_ERR_SHAPE before any launch.
@@ -339,8 +339,11 @@ QKN_API qkn_status qkv_norm_proj(const void *x, const void *W_folded, void *y,
  *   caller.  Each call writes the entries it reads, so the array's leftover
  *   contents from an earlier call never reach the result.
  * - The first call on a device (with that device current) looks up the
- *   array's device address with cudaGetSymbolAddress and caches it; make that
- *   first call before any stream capture.
+ *   array's device address with cudaGetSymbolAddress and caches it with the
+ *   current CUDA context; make that first call before any stream capture.
+ *   If the context changes (e.g. after cudaDeviceReset the module is loaded
+ *   again, possibly elsewhere), the next call looks the address up again, so
+ *   that call, too, belongs outside a stream capture.
  */
 QKN_API qkn_status flashnorm_proj_noalloc(const void *x, const void *W_folded, void *y,
                                           int64_t M, int64_t N, int64_t K, int w_k_major,

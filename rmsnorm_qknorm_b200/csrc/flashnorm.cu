@@ -14,6 +14,8 @@
 #include <math.h>
 
 #include <mutex>
+#include <stdlib.h>
+#include <string.h>
 
 #include "gemm_tc.cuh"
 #include "qkn_common.cuh"
@@ -243,7 +245,8 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
     uint64_t *stats_full = bars + 2 * STAGES + 4;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 6);
+    uint64_t *drained = bars + 2 * STAGES + 6;  // every MMA this CTA issued has completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 7);
     float *inv_buf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES);  // [2][BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -259,6 +262,7 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             mbar_init(smem_u32(&acc_empty[a]), 4);   // one arrive per epilogue warp
             mbar_init(smem_u32(&stats_full[a]), 2);  // one arrive per statistics warp
         }
+        mbar_init(smem_u32(drained), 1);             // the MMA warp's final tcgen05.commit
         mbar_init_fence();
     }
     if (warp == 1) {  // whole warp: allocate the two accumulators in tensor memory
@@ -275,6 +279,7 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
         // ---------------------------------------------------------------- TMA producer
         int stage = 0;
         uint32_t phase = 0;
+        uint32_t armed = 0, armed_parity = 0;  // per stage: loads issued; parity of the phase they complete
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
             int m_blk, n_blk;
@@ -288,10 +293,20 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
                     tma_load_2d(smem_u32(sa), &tmap_x, kb * BK, m_blk * BM, fb);
                     tma_load_2d(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, n_blk * BN, fb);
                 }
+                armed |= 1u << stage;
+                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
                 __syncwarp();
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
         }
+        // No copy may still be writing shared memory when the CTA exits: wait
+        // (bounded) for the last phase armed on every stage.  On the normal
+        // path the MMA warp consumed them all and these return at once; after
+        // a wait gave up they catch loads nobody will consume.
+        if (lane == 0)
+            for (int s2 = 0; s2 < STAGES; ++s2)
+                if (armed & (1u << s2)) mbar_wait(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, &g_device_error);
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         int stage = 0;
@@ -325,6 +340,13 @@ flashnorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_c
             if (lane == 0) umma_commit(smem_u32(&acc_full[acc]));  // accumulator ready
             __syncwarp();
         }
+        // Tensor memory is released only after every MMA issued here has
+        // completed, also when a wait above gave up with MMAs in flight.
+        if (lane == 0) {
+            umma_commit(smem_u32(drained));
+            mbar_wait(smem_u32(drained), 0u, &g_device_error);
+        }
+        __syncwarp();
     } else if (warp < 6) {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
         // Launched right behind the statistics pass (programmatic dependent
@@ -527,6 +549,20 @@ qkn_status launch_inv_rms(const void *x, float *inv, int64_t M, int64_t K, float
     return check_launch("inv_rms_kernel launch");
 }
 
+#include "gemm_pair.cuh"
+
+// Which projection kernel serves the calls with a given 1/rms (or none):
+// QKN_GEMM_KERNEL=pair selects the CTA-pair kernel, =single the single-CTA
+// one; otherwise the default below.  Read on every call (a getenv), so a
+// process can compare both.  The in-kernel statistics form always runs on
+// the single-CTA kernel.
+bool use_pair_kernel() {
+    const char *v = getenv("QKN_GEMM_KERNEL");
+    if (v != nullptr && strcmp(v, "pair") == 0) return true;
+    if (v != nullptr && strcmp(v, "single") == 0) return false;
+    return false;
+}
+
 namespace {
 
 // inv == nullptr (and not unit_scale): the single-CTA kernel computes every
@@ -555,6 +591,8 @@ qkn_status launch_gemm(const void *x, const void *Wf, void *y, const float *inv,
     g.n_blocks = (int)((N + gemm::BN - 1) / gemm::BN);
     g.k_blocks = (int)((K + gemm::BK - 1) / gemm::BK);
     g.num_tiles = g.m_blocks * g.n_blocks;
+    if (!g.compute_inv && use_pair_kernel() && sm_count() >= 2)
+        return launch_gemm_pair(x, Wf, y, inv, M, N, K, unit_scale, s, after_stats);
     static std::atomic<bool> attr_set[64];  // per device: the attribute has been set
     int dev = 0;
     cudaGetDevice(&dev);
@@ -674,8 +712,10 @@ extern "C" QKN_API qkn_status flashnorm_proj(const void *x, const void *W_folded
         // the caller's buffer is the workspace of a separate row-statistics
         // pass, which leaves the matmul's shared-memory bandwidth to the MMA
         st = launch_inv_rms(x, inv_rms_out, M, K, eps, s);
-        // FlashNorm's "RMS and matmul in parallel": the projection starts while
-        // the statistics pass runs and waits for it only in its epilogue
+        // FlashNorm (abstract, item (ii)): with the scaling deferred, the row
+        // statistic and the matmul can run at the same time, so the projection
+        // starts while the statistics pass runs and waits for it only in its
+        // epilogue
         if (st == QKN_OK) st = launch_gemm(x, Wk, y, inv_rms_out, M, N, K, eps, nullptr, s, false, true);
     } else {
         // with no 1/rms at all the GEMM computes it beside the matmul (no workspace)
@@ -722,9 +762,11 @@ extern "C" QKN_API qkn_status qkn_check_device(void *stream) {
 // GPU shares it, so calls that overlap on the GPU race on it.  Each call
 // overwrites the entries it uses before reading them, so nothing has to start
 // at zero.  In host code the name g_noalloc_inv_rms is only a host-side
-// stand-in; its device address is fetched once per device with
-// cudaGetSymbolAddress (on the first call made with that device current) and
-// cached.
+// stand-in; its device address is fetched with cudaGetSymbolAddress on the
+// first call made with a device current and cached together with the CUDA
+// context it belongs to.  A later call that finds another context current on
+// that device (the primary context was reset and the module loaded again,
+// possibly at another address) fetches the address again.
 
 namespace qkn {
 namespace {
@@ -735,23 +777,52 @@ static __device__ __align__(256) float g_noalloc_inv_rms[kNoAllocMaxRows];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-float *g_noalloc_ptr[kMaxDevices] = {nullptr};
+struct NoAllocSlot {
+    CUcontext ctx;  // context the cached address belongs to
+    float *ptr;
+};
+NoAllocSlot g_noalloc_slot[kMaxDevices] = {};
 
-// Device address of g_noalloc_inv_rms on the current device (set up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+// The driver's cuCtxGetCurrent, looked up once through the runtime (the
+// library does not link libcuda directly).
+CtxGetCurrentFn ctx_get_current_fn() {
+    static const CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<CtxGetCurrentFn>(p);
+        return nullptr;
+    }();
+    return fn;
+}
+
+// Device address of g_noalloc_inv_rms in the current device's current context.
 qkn_status noalloc_scratch(float **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "flashnorm_proj_noalloc: cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(QKN_ERR_UNSUPPORTED, "flashnorm_proj_noalloc: device %d", dev);
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return fail(QKN_ERR_CUDA, "flashnorm_proj_noalloc: cuCtxGetCurrent is unavailable");
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return fail(QKN_ERR_CUDA, "flashnorm_proj_noalloc: cuCtxGetCurrent failed");
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    NoAllocSlot &slot = g_noalloc_slot[dev];
+    if (slot.ptr == nullptr || ctx == nullptr || slot.ctx != ctx) {
+        // also makes the runtime bind the device's primary context when none was current yet
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_inv_rms);
         if (e != cudaSuccess || p == nullptr)
             return cuda_fail(e, "flashnorm_proj_noalloc: cudaGetSymbolAddress(scratch)");
-        g_noalloc_ptr[dev] = static_cast<float *>(p);
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+            return fail(QKN_ERR_CUDA, "flashnorm_proj_noalloc: no current context after the symbol lookup");
+        slot.ctx = ctx;
+        slot.ptr = static_cast<float *>(p);
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return QKN_OK;
 }
 

@@ -129,14 +129,38 @@ qkn_status launch_vec(RowArgs &a, int njobs, cudaStream_t s) {
     return check_launch("rownorm_vec_kernel launch");
 }
 
-template <typename TA, typename TW, bool STATS>
+template <typename TA, typename TW, bool STATS, bool MANY = false>
 qkn_status launch_vec_stream(RowArgs &a, int njobs, cudaStream_t s) {
     int64_t groups = 0;
     for (int i = 0; i < njobs; ++i) groups += a.job[i].nblocks;
     const int64_t cap = 2 * (int64_t)sm_count();  // two 256-thread blocks per SM
     const unsigned grid = (unsigned)(groups < cap ? groups : cap);
-    rownorm_vec_stream_kernel<TA, TW, STATS><<<grid, stream::BLOCK, 0, s>>>(a);
+    rownorm_vec_stream_kernel<TA, TW, STATS, MANY><<<grid, stream::BLOCK, 0, s>>>(a);
     return check_launch("rownorm_vec_stream_kernel launch");
+}
+
+// Job geometry of the register kernels: a row in 2^tpr_log2 threads of `cpt`
+// chunks each, `block` threads per CTA.
+template <typename TA>
+void setup_vec_jobs(RowArgs &a, const Tensor2 *ts, int njobs, int64_t rows, int n_seg, int cpt, int block) {
+    constexpr int E = Chunk<TA>::E;
+    for (int i = 0; i < njobs; ++i) {
+        const Tensor2 &t = ts[i];
+        RowJob &J = a.job[i];
+        J.x = static_cast<const uint8_t *>(t.x);
+        J.y = static_cast<uint8_t *>(t.y);
+        J.w = t.w;
+        J.ld_bytes = t.ld * (int64_t)sizeof(TA);
+        J.ldo_bytes = t.ldo * (int64_t)sizeof(TA);
+        J.rows = rows;
+        J.d = (int)t.d;
+        J.nchunks = (int)(t.d / E);
+        J.seg_chunks = J.nchunks / n_seg;
+        J.inv_seg_chunks = 1.0f / (float)J.seg_chunks;
+        J.tpr_log2 = ceil_log2((J.nchunks + cpt - 1) / cpt);
+        J.rows_per_cta = block >> J.tpr_log2;
+        J.nblocks = (rows + J.rows_per_cta - 1) / J.rows_per_cta;
+    }
 }
 
 // Ring geometry for the staged kernel: stage = the widest row (rounded up to
@@ -342,6 +366,13 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
     // More than 8 segments (the register kernel stops at 8) take the staged
     // kernel's many-segment statistic when its ring holds the rows.
     const bool many = chunked && n_seg > kFastMaxSeg;
+    // Rows of at most 4 KiB with 9-64 segments: the streaming register kernel
+    // with its many-segment statistic (per-chunk sums parked in shared memory,
+    // each segment added in chunk order by one lane).
+    if (many && max_chunks <= 32 * stream::CPT && max_row_bytes <= kRegisterMaxRowBytes) {
+        setup_vec_jobs<TA>(a, ts, njobs, rows, n_seg, stream::CPT, stream::BLOCK);
+        return launch_vec_stream<TA, TW, STATS, true>(a, njobs, s);
+    }
     if ((vec && max_row_bytes > (STATS ? kRegisterMaxRowBytesStats : kRegisterMaxRowBytes)) || many) {
         int64_t w_bytes = 0;
         for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
@@ -353,24 +384,7 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
     }
 
     if (vec) {
-        const int cpt = kVecCfgs[cfg].cpt, block = kVecCfgs[cfg].block;
-        for (int i = 0; i < njobs; ++i) {
-            const Tensor2 &t = ts[i];
-            RowJob &J = a.job[i];
-            J.x = static_cast<const uint8_t *>(t.x);
-            J.y = static_cast<uint8_t *>(t.y);
-            J.w = t.w;
-            J.ld_bytes = t.ld * (int64_t)sizeof(TA);
-            J.ldo_bytes = t.ldo * (int64_t)sizeof(TA);
-            J.rows = rows;
-            J.d = (int)t.d;
-            J.nchunks = (int)(t.d / E);
-            J.seg_chunks = J.nchunks / n_seg;
-            J.inv_seg_chunks = 1.0f / (float)J.seg_chunks;
-            J.tpr_log2 = ceil_log2((J.nchunks + cpt - 1) / cpt);
-            J.rows_per_cta = block >> J.tpr_log2;
-            J.nblocks = (rows + J.rows_per_cta - 1) / J.rows_per_cta;
-        }
+        setup_vec_jobs<TA>(a, ts, njobs, rows, n_seg, kVecCfgs[cfg].cpt, kVecCfgs[cfg].block);
         // narrow rows (at most 32 threads per row) stream through persistent
         // blocks that load the next rows while they normalise the current ones
         // (the statistics alone keep the one-shot form, which measured as fast

@@ -166,7 +166,8 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *acc_full = bars + 2 * STAGES, *acc_empty = bars + 2 * STAGES + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+    uint64_t *drained = bars + 2 * STAGES + 4;  // every MMA this CTA issued has completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -179,6 +180,7 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             mbar_init(smem_u32(&acc_full[a]), 1);   // one tcgen05.commit
             mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrive per epilogue warp
         }
+        mbar_init(smem_u32(drained), 1);            // the MMA warp's final tcgen05.commit
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -195,6 +197,7 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
         // ---------------------------------------------------------------- TMA producer
         int stage = 0;
         uint32_t phase = 0;
+        uint32_t armed = 0, armed_parity = 0;  // per stage: loads issued; parity of the phase they complete
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
             const Tile t = tile_of(tile, g);
@@ -207,10 +210,20 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                     tma_load_2d(smem_u32(sa), &tmap_x, kb * BK, t.m_blk * BM, fb);
                     tma_load_2d(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, t.col0, fb);
                 }
+                armed |= 1u << stage;
+                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
                 __syncwarp();
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
         }
+        // No copy may still be writing shared memory when the CTA exits: wait
+        // (bounded) for the last phase armed on every stage (immediate on the
+        // normal path, where the MMA warp consumed them all).
+        if (lane == 0)
+            for (int s2 = 0; s2 < STAGES; ++s2)
+                if (armed & (1u << s2))
+                    mbar_wait(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, &g_qkv_error, g.wait_ns);
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         int stage = 0;
@@ -242,6 +255,13 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             if (lane == 0) gemm::umma_commit(smem_u32(&acc_full[acc]));
             __syncwarp();
         }
+        // Tensor memory is released only after every MMA issued here has
+        // completed, also when a wait above gave up with MMAs in flight.
+        if (lane == 0) {
+            gemm::umma_commit(smem_u32(drained));
+            mbar_wait(smem_u32(drained), 0u, &g_qkv_error, g.wait_ns);
+        }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
         const int quarter = warp & 3;  // TMEM lanes 32 * quarter ... of the accumulator

@@ -188,6 +188,15 @@ namespace stream {
 
 constexpr int CPT = 8;
 constexpr int BLOCK = 256;
+// Many-segment statistic (9 to QKN_MAX_SEG segments): per warp, the chunk
+// sums of its rows (32 x CPT slots, one padding float after every 32 so that
+// lanes summing neighbouring segments read distinct banks) and the segment
+// sums (at most 32 x CPT of them: a row of n_seg segments holds at least
+// n_seg chunks).
+constexpr int kChunkSlots = 32 * CPT + 32 * CPT / 32;
+constexpr int kScratchPerWarp = kChunkSlots + 32 * CPT;
+
+__device__ __forceinline__ int padded(int i) { return i + (i >> 5); }
 
 template <typename TA>
 __device__ __forceinline__ void load_group(const RowArgs &a, int64_t g, int64_t n0, uint4 (&v)[CPT]) {
@@ -205,6 +214,77 @@ __device__ __forceinline__ void load_group(const RowArgs &a, int64_t g, int64_t 
         if (active && c < J.nchunks) v[i] = ld_stream(xr + (int64_t)c * 16);
         else v[i] = make_uint4(0u, 0u, 0u, 0u);
     }
+}
+
+// Normalises (or, STATS, writes the segment sums of) the rows of a group
+// from the n_seg > 8 segment sums formed in shared memory: every thread
+// parks the sum of squares of each of its chunks, lane k of the warp then
+// adds the chunks of segment k % n_seg of row k / n_seg in chunk order (and
+// k + 32, ...), and the row's statistic combines its segment sums left to
+// right.  The order of every sum is fixed by the row width and n_seg alone.
+template <typename TA, typename TW, bool STATS>
+__device__ __forceinline__ void process_group_many(const RowArgs &a, const RowJob &J, int64_t b,
+                                                   const uint4 (&v)[CPT], float *scratch) {
+    constexpr int E = Chunk<TA>::E;
+    const int lane = threadIdx.x & 31;
+    const int tpr = 1 << J.tpr_log2;
+    const int t = threadIdx.x & (tpr - 1);
+    const int rloc = lane >> J.tpr_log2;           // row within the warp
+    const int rpw = 32 >> J.tpr_log2;              // rows per warp
+    const int cap = tpr * CPT;                     // chunk slots per row
+    const int64_t row0 = b * J.rows_per_cta + (int64_t)(threadIdx.x >> 5) * rpw;  // the warp's first row
+    const int64_t row = row0 + rloc;
+    const bool active = row < J.rows;
+    const int nchunks = J.nchunks, n_seg = a.n_seg, sc = J.seg_chunks;
+    float *cs = scratch;                           // chunk sums, padded
+    float *ss = scratch + kChunkSlots;             // segment sums [rpw][n_seg]
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * tpr + t;
+        float f[E];
+        Chunk<TA>::unpack(v[i], f);
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+        if (c < nchunks) cs[padded(rloc * cap + c)] = s;
+    }
+    __syncwarp();
+    const int tasks = rpw * n_seg;
+    for (int k = lane; k < tasks; k += 32) {
+        const int r = k / n_seg, j = k - r * n_seg;
+        const int base = r * cap + j * sc;
+        float s = 0.f;
+        for (int q = 0; q < sc; ++q) s += cs[padded(base + q)];
+        ss[k] = s;
+    }
+    __syncwarp();
+    if constexpr (STATS) {
+        for (int k = lane; k < tasks; k += 32) {
+            const int r = k / n_seg;
+            if (row0 + r < J.rows) a.partial[(row0 + r) * n_seg + (k - r * n_seg)] = ss[k];
+        }
+    } else {
+        float S = 0.f;
+        if (t == 0)
+            for (int j = 0; j < n_seg; ++j) S += ss[rloc * n_seg + j];
+        S = __shfl_sync(0xffffffffu, S, rloc << J.tpr_log2);
+        const float inv = rsqrtf(S / (float)J.d + a.eps);
+        uint8_t *yr = J.y + (active ? row : 0) * J.ldo_bytes;
+        const TW *w = static_cast<const TW *>(J.w);
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = i * tpr + t;
+            if (active && c < nchunks) {
+                float f[E], wf[E];
+                Chunk<TA>::unpack_again(v[i], f);
+                load_weights<TW, E>(w + (int64_t)c * E, wf);
+#pragma unroll
+                for (int e = 0; e < E; ++e) f[e] = (f[e] * inv) * wf[e];
+                st_stream(yr + (int64_t)c * 16, Chunk<TA>::pack(f));
+            }
+        }
+    }
+    __syncwarp();  // the next group rewrites the scratch
 }
 
 template <typename TA, typename TW, bool STATS>
@@ -273,17 +353,25 @@ __device__ __forceinline__ void process_group(const RowArgs &a, int64_t g, int64
 
 }  // namespace stream
 
-template <typename TA, typename TW, bool STATS>
+// MANY: n_seg of 9 to QKN_MAX_SEG (rows of at most 32 x CPT chunks).
+template <typename TA, typename TW, bool STATS, bool MANY>
 __global__ void __launch_bounds__(stream::BLOCK, 2) rownorm_vec_stream_kernel(const RowArgs a) {
     const int64_t n0 = a.job[0].nblocks, total = n0 + a.job[1].nblocks;
     int64_t g = blockIdx.x;
     if (g >= total) return;  // the whole block: no block-level synchronisation below
+    __shared__ float scratch[MANY ? stream::BLOCK / 32 * stream::kScratchPerWarp : 1];
     uint4 cur[stream::CPT], nxt[stream::CPT];
     stream::load_group<TA>(a, g, n0, cur);
     for (; g < total; g += gridDim.x) {
         const int64_t gn = g + gridDim.x;
         if (gn < total) stream::load_group<TA>(a, gn, n0, nxt);
-        stream::process_group<TA, TW, STATS>(a, g, n0, cur);
+        if constexpr (MANY) {
+            const int which = g >= n0 ? 1 : 0;
+            stream::process_group_many<TA, TW, STATS>(a, pick_job(a, which), g - (which ? n0 : 0), cur,
+                                                      scratch + (threadIdx.x >> 5) * stream::kScratchPerWarp);
+        } else {
+            stream::process_group<TA, TW, STATS>(a, g, n0, cur);
+        }
 #pragma unroll
         for (int i = 0; i < stream::CPT; ++i) cur[i] = nxt[i];
     }

@@ -29,6 +29,12 @@ def test_reference_arm_json_line(workload):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["ms_per_step"] > 0
+    # the same metric string as the GPU arm's line for this workload, so the two lines compare
+    sys.path.insert(0, ROOT)
+    import bench
+    expected = {"tiny": bench.METRIC_QK, "qkv_proj_qknorm": bench.METRIC_QKV, "tp_qknorm": bench.METRIC_TP}
+    assert d["metric"] == expected[workload]
 
 
 def test_reference_arm_other_ranks_exit_quietly():

@@ -9,8 +9,8 @@ to the host exactly:
 
 Sizes: every workload at oracle-friendly sizes that span several blocks with a
 ragged tail, the two small workloads at full size, and the two large ones at
-full size in the exact launch configuration the benchmark times, checked on
-sampled rows plus properties that hold for every row.
+full size in the exact launch configuration the benchmark times, every row
+checked against the oracle.
 """
 from __future__ import annotations
 
@@ -55,8 +55,13 @@ def test_workload_parity_oracle_sized(cuda_lib, name, tokens):
     check(ko, inp["k"], inp["wk"], inp["eps"], f"{name} k")
 
 
-def _full_size_sampled(name, n_sample=384):
+def _full_size_all_rows(name, chunk=8192, parts=5):
+    """The workload at full size in the benchmark's launch configuration: every
+    row of q and k against the oracle (in chunks of rows, so the fp64 copies
+    stay small), determinism, and the same rows normalised by several shorter
+    launches giving the same bits as the one long launch."""
     wl = W.QKNORM_WORKLOADS[name]
+    T = wl.tokens
     inp = W.make_qknorm_inputs(name, seed=0, device=DEV)
     qo, ko = run_pair(inp)
     qo2, ko2 = run_pair(inp)
@@ -64,24 +69,26 @@ def _full_size_sampled(name, n_sample=384):
     # determinism: bitwise-equal outputs on a second call
     assert torch.equal(qo.view(torch.int16), qo2.view(torch.int16))
     assert torch.equal(ko.view(torch.int16), ko2.view(torch.int16))
-    g = torch.Generator().manual_seed(7)
-    rows = torch.unique(torch.cat([torch.tensor([0, 1, wl.tokens - 2, wl.tokens - 1]),
-                                   torch.randint(0, wl.tokens, (n_sample,), generator=g)]))
-    rd = rows.to(DEV)
-    check(qo[rd], inp["q"][rd], inp["wq"], wl.eps, f"{name} q sampled")
-    check(ko[rd], inp["k"][rd], inp["wk"], wl.eps, f"{name} k sampled")
-    # every row: finite, and (y / w) has unit mean square up to bf16 rounding
-    for y, w in ((qo, inp["wq"]), (ko, inp["wk"])):
-        z = y.float() / w.float()
-        ms = z.pow(2).mean(dim=1)
-        assert torch.isfinite(y.float()).all()
-        assert (ms - 1).abs().max().item() < 2e-2
+    del qo2, ko2
+    # the same rows in `parts` shorter launches of unequal length (ragged ends)
+    cuts = sorted({0, T} | {int(T * f) + 1 for f in (0.13, 0.4, 0.41, 0.77)[:parts - 1]})
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        qs, ks = qk.qknorm_fused(inp["q"][a:b], inp["k"][a:b], inp["wq"], inp["wk"], wl.eps, wl.n_seg)
+        torch.cuda.synchronize()
+        assert torch.equal(qs.view(torch.int16), qo[a:b].view(torch.int16)), f"{name} q rows {a}:{b}"
+        assert torch.equal(ks.view(torch.int16), ko[a:b].view(torch.int16)), f"{name} k rows {a}:{b}"
+    # every row against the oracle
+    wq, wk = inp["wq"].cpu(), inp["wk"].cpu()
+    for r0 in range(0, T, chunk):
+        r1 = min(T, r0 + chunk)
+        check(qo[r0:r1], inp["q"][r0:r1], wq, wl.eps, f"{name} q rows {r0}:{r1}")
+        check(ko[r0:r1], inp["k"][r0:r1], wk, wl.eps, f"{name} k rows {r0}:{r1}")
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["prefill_gqa", "long_context", "narrow_rows"])
 def test_workload_parity_full_size(cuda_lib, name):
-    _full_size_sampled(name)
+    _full_size_all_rows(name)
 
 
 # ------------------------------------------------------------------ n_seg coverage
@@ -293,9 +300,11 @@ def test_register_kernel_many_rows(cuda_lib, dq, dk, n_seg):
 @pytest.mark.parametrize("dq,dk,n_seg", [(4096, 1024, 16), (5120, 1024, 64), (5120, 5120, 40), (2048, 256, 32),
                                          (1024, 128, 16)])
 def test_many_segments_staged(cuda_lib, dtype, dq, dk, n_seg):
-    # 9 .. 64 segments through the staged kernel's many-segment statistic: segments of
-    # 2 chunks (lanes skip segments), a count that is not a power of two, ragged T;
-    # the partial sums themselves, and the same bits from a short launch
+    # 9 .. 64 segments: rows wider than 4 KiB through the staged kernel's many-segment
+    # statistic (segments of 2 chunks: lanes skip segments; a count that is not a
+    # power of two), narrower launches (2048 + 256 and 1024 + 128 bf16) through the
+    # streaming register kernel's; ragged T, the partial sums themselves, and the same
+    # bits from a short launch
     if dtype == torch.float32 and (dq // n_seg) % 4:
         pytest.skip("segments not whole fp32 chunks")
     T = 301
@@ -330,6 +339,36 @@ def test_register_stream_many_groups(cuda_lib, T, dq, dk):
     check(ko[rows], inp["k"][rows], inp["wk"], inp["eps"], f"k T={T} d={dk}")
     assert torch.equal(qo[-300:].view(torch.int16), qs.view(torch.int16))
     assert torch.equal(ko[-300:].view(torch.int16), ks.view(torch.int16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dq,dk,n_seg", [(128, 128, 16), (256, 512, 32), (512, 512, 64), (1024, 128, 16),
+                                         (1024, 1024, 64), (2048, 256, 32)])
+def test_register_stream_many_segments(cuda_lib, dtype, dq, dk, n_seg):
+    # rows of at most 4 KiB with 9 .. 64 segments: the streaming register kernel's
+    # many-segment statistic (chunk sums parked in shared memory, each segment added
+    # in chunk order); several row groups per persistent block, a ragged last group,
+    # every row against the oracle, the partial sums, a short launch bit for bit
+    if (dq * dtype.itemsize > 4096 or dk * dtype.itemsize > 4096
+            or (dk // n_seg) * dtype.itemsize % 16 or (dq // n_seg) * dtype.itemsize % 16):
+        pytest.skip("rows wider than 4 KiB or segments not whole 16-byte chunks")
+    T = 20001
+    g = torch.Generator().manual_seed(dq + dk + n_seg)
+    q = (torch.randn(T, dq, generator=g) * 2).to(dtype).to(DEV)
+    k = torch.randn(T, dk, generator=g).to(dtype).to(DEV)
+    wq = (1 + 0.1 * torch.randn(dq, generator=g)).to(dtype).to(DEV)
+    wk = (1 + 0.1 * torch.randn(dk, generator=g)).to(dtype).to(DEV)
+    qo, ko = qk.qknorm_fused(q, k, wq, wk, 1e-6, n_seg)
+    qs, ks = qk.qknorm_fused(q[-77:], k[-77:], wq, wk, 1e-6, n_seg)
+    pq = qk.rmsnorm_partial_stats(q, n_seg)
+    pk = qk.rmsnorm_partial_stats(k[:333], n_seg)
+    torch.cuda.synchronize()
+    check(qo, q, wq, 1e-6, f"q d={dq} n_seg={n_seg}")
+    check(ko, k, wk, 1e-6, f"k d={dk} n_seg={n_seg}")
+    bits = (lambda t: t.view(torch.int16)) if dtype == torch.bfloat16 else (lambda t: t)
+    assert torch.equal(bits(qo[-77:]), bits(qs)) and torch.equal(bits(ko[-77:]), bits(ks))
+    assert_f32_close(pq, oracle.segment_partials(q.cpu(), n_seg), tol=PARTIAL_REL_TOL, what="q partials")
+    assert_f32_close(pk, oracle.segment_partials(k[:333].cpu(), n_seg), tol=PARTIAL_REL_TOL, what="k partials")
 
 
 @pytest.mark.parametrize("act,wdt", [(torch.float32, torch.float32), (torch.bfloat16, torch.float32),

@@ -126,8 +126,10 @@ def test_matches_two_step_device_path(cuda_lib):
 
 
 @pytest.mark.slow
-def test_full_size_sampled(cuda_lib):
-    # x [8192, 4096] with W [4096, 12288] split q | k | v = 4096 each, sampled rows vs the oracle
+def test_full_size_every_row_block(cuda_lib):
+    # x [8192, 4096] with W [4096, 12288] split q | k | v = 4096 each: one row of every
+    # 128-row tile block (and the last row), all N columns, against the oracle
+    from test_flashnorm_gpu import block_rows
     wl = W.FLASHNORM_WORKLOAD
     nq = nk = nv = wl.N // 3
     inp = W.make_flashnorm_inputs(seed=0, device=DEV)
@@ -137,13 +139,12 @@ def test_full_size_sampled(cuda_lib):
     Wf = qk.flashnorm_fold_weights(inp["w"], inp["W"])
     y = qk.qkv_proj_qknorm(inp["x"], Wf, nq, nk, nv, wq.to(DEV), wk.to(DEV), wl.eps)
     torch.cuda.synchronize()
-    rows = torch.unique(torch.cat([torch.tensor([0, 127, 128, wl.M - 1]),
-                                   torch.randint(0, wl.M, (20,), generator=g)]))
-    xs = inp["x"][rows.to(DEV)].cpu()
+    rows = block_rows(wl.M, seed=4)
+    rd = rows.to(DEV)
+    xs = inp["x"][rd].cpu()
     ref = oracle.qkv_proj_qknorm(xs, inp["w"].cpu(), inp["W"].cpu(), wq, wk, nq, nk, wl.eps, wl.eps)
-    ys = y[rows.to(DEV)].cpu()
-    for name, lo, hi in _sections(nq, nk, nv):
-        err = frobenius_rel(ys[:, lo:hi], ref[:, lo:hi])
-        assert err <= PROJ_FROB_TOL, f"full size {name}: {err:.3e}"
+    ref_used = oracle.qkv_proj_qknorm(xs, torch.ones(wl.K), Wf.float().cpu().T.contiguous(), wq, wk, nq, nk,
+                                      wl.eps, wl.eps)
+    _check(y[rd], ref, ref_used, nq, nk, nv, "full size, one row per 128-row block")
     assert torch.isfinite(y.float()).all()
     assert qk.load_library().qkn_check_device(None) == 0, qk.load_library().qkn_last_error()

@@ -4,10 +4,13 @@ Some callers must not allocate device memory while they run (runtimes that
 pre-plan every byte of the GPU, callers whose framework owns the allocator,
 latency-critical loops).  The no-allocation entry point keeps the 1/rms
 scratch in a fixed array compiled into the library.  This test calls it
-through the C ABI and checks it against the allocating entry point,
-flashnorm_proj, on two calls in a row with different inputs and sizes (the
-second call must not see the first call's scratch), and that an M beyond the
-fixed array is rejected before any launch.
+through the C ABI on two calls in a row with different inputs and sizes and
+checks each result bit for bit against the allocating entry point,
+flashnorm_proj (the same two kernels), and against the fp64 oracle.  The
+second call's rows have a 1/rms three orders of magnitude away from the
+first's, so a scratch entry left over from the first call cannot go
+unnoticed.  It also checks that an M beyond the fixed array is rejected
+before any launch.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -40,21 +43,38 @@ def _noalloc_fn():
 def test_noalloc_matches_allocating_entry_point():
     if not torch.cuda.is_available():
         pytest.fail("GPU test collected on a machine without CUDA")
+    import oracle
+    from parity import frobenius_rel
     lib, f = _noalloc_fn()
     stream = torch.cuda.current_stream().cuda_stream
-    # two calls in a row: a larger problem, then a smaller one on different data
-    for seed, (M, K, N) in ((0, (1000, 512, 776)), (1, (257, 1024, 264))):
+    # Two calls in a row on different data and sizes.  The second call's rows
+    # alternate between N(0,1) and N(0,1) x 1000, so their 1/rms differ from
+    # the first call's (~1) by three orders of magnitude: an entry of the
+    # shared scratch left over from call 1 would make that row of call 2
+    # wrong by a factor of ~1000, not by a few percent.
+    for call, (seed, (M, K, N), scale) in enumerate(((0, (1000, 512, 776), False),
+                                                     (1, (777, 1024, 264), True))):
         inp = W.make_flashnorm_inputs(seed=seed, M=M, K=K, N=N)
-        x = inp["x"].to(DEV)
+        x_host = inp["x"]
+        if scale:
+            x_host = x_host.float()
+            x_host[1::2] *= 1000.0
+            x_host = x_host.to(torch.bfloat16)
+        x = x_host.to(DEV)
         Wf = qk.flashnorm_fold_weights(inp["w"].to(DEV), inp["W"].to(DEV))
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
         st = f(x.data_ptr(), Wf.data_ptr(), y.data_ptr(), M, N, K, 1, inp["eps"], stream)
         assert st == 0, lib.qkn_last_error().decode()
-        y_ref = qk.flashnorm_proj(x, Wf, inp["eps"])  # the allocating entry point
+        # the allocating entry point: the same statistics pass and projection
+        y_ref = qk.flashnorm_proj(x, Wf, inp["eps"])
         torch.cuda.synchronize()
-        ref = y_ref.double()
-        err = ((y.double() - ref).norm() / ref.norm()).item()
-        assert err <= PROJ_FROB_TOL, f"call {seed}: relative Frobenius error {err:.3e}"
+        same = y.view(torch.int16) == y_ref.view(torch.int16)
+        assert bool(same.all()), (f"call {call}: {int((~same).sum())} of {same.numel()} outputs differ from "
+                                  f"flashnorm_proj; first rows {torch.nonzero(~same)[:4, 0].tolist()}")
+        # and the result itself against the fp64 oracle (original w and W)
+        ref = oracle.norm_then_project(x_host, inp["w"], inp["W"], inp["eps"])
+        err = frobenius_rel(y, ref)
+        assert err <= PROJ_FROB_TOL, f"call {call}: relative Frobenius error {err:.3e} against the oracle"
     assert lib.qkn_check_device(None) == 0, lib.qkn_last_error()
 
 

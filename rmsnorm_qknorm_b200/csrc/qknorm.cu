@@ -135,7 +135,20 @@ qkn_status launch_vec_stream(RowArgs &a, int njobs, cudaStream_t s) {
     for (int i = 0; i < njobs; ++i) groups += a.job[i].nblocks;
     const int64_t cap = 2 * (int64_t)sm_count();  // two 256-thread blocks per SM
     const unsigned grid = (unsigned)(groups < cap ? groups : cap);
-    rownorm_vec_stream_kernel<TA, TW, STATS, MANY><<<grid, stream::BLOCK, 0, s>>>(a);
+    // programmatic dependent launch: back-to-back launches overlap one's
+    // last blocks with the next one's start (the kernel waits for the
+    // previous grid before its first global access)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(stream::BLOCK, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, rownorm_vec_stream_kernel<TA, TW, STATS, MANY>, a);
+    if (e != cudaSuccess) return cuda_fail(e, "rownorm_vec_stream_kernel launch");
     return check_launch("rownorm_vec_stream_kernel launch");
 }
 

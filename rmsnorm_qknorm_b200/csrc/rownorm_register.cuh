@@ -356,6 +356,12 @@ __device__ __forceinline__ void process_group(const RowArgs &a, int64_t g, int64
 // MANY: n_seg of 9 to QKN_MAX_SEG (rows of at most 32 x CPT chunks).
 template <typename TA, typename TW, bool STATS, bool MANY>
 __global__ void __launch_bounds__(stream::BLOCK, 2) rownorm_vec_stream_kernel(const RowArgs a) {
+    // Launched as the programmatic dependent of the previous launch on the
+    // stream: let the next launch's blocks take SM slots as this grid's
+    // blocks exit, and touch global memory only once the previous grid has
+    // completed and its writes are visible.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t n0 = a.job[0].nblocks, total = n0 + a.job[1].nblocks;
     int64_t g = blockIdx.x;
     if (g >= total) return;  // the whole block: no block-level synchronisation below

@@ -2,15 +2,16 @@
 //
 // Included by flashnorm.cu (it shares that file's device error word).
 //
-// Why a pair: the single-CTA kernel multiplies a 128 x 64 x tile by a
-// 256 x 64 W' tile per k-block, 48 KiB brought from L2 into shared memory
-// for 2M multiply-adds -- more operand bytes per clock than L2 delivers to
-// an SM, so its tensor pipe idles about a quarter of the time.  Two CTAs of
-// a cluster (the two SMs of a TPC) computing one 256 x 256 tile with
-// tcgen05.mma.cta_group::2 need a third less: each CTA loads only its own
-// 128 x rows and its own 128 W' rows (32 KiB per k-block), the MMA reads
-// both CTAs' tiles, and each CTA's tensor memory holds the fp32 accumulator
-// of its own 128 rows over all 256 columns.
+// The default kernel of the projection (the single-CTA kernel in
+// flashnorm.cu serves the in-kernel statistics form).  Two CTAs of a
+// cluster (the two SMs of a TPC) compute one 256 x 256 tile with
+// tcgen05.mma.cta_group::2: each CTA loads only its own 128 x rows and its
+// own 128 W' rows (32 KiB per k-block instead of the single-CTA kernel's
+// 48 KiB), the MMA reads both CTAs' tiles, and each CTA's tensor memory
+// holds the fp32 accumulator of its own 128 rows over all 256 columns.  The
+// smaller stages give a 6-deep ring: what limits these kernels is the round
+// trip a stage makes (MMAs complete, commit, refill, next MMAs), and a
+// deeper ring hides more of it.
 //
 // Roles (192 threads per CTA):
 //   warp 0     TMA producer, both CTAs: this CTA's x and W' tiles of a stage
@@ -136,43 +137,45 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer (both CTAs)
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t armed = 0, armed_parity = 0;  // per stage: loads issued; parity of the phase they complete
-        bool ok = true;
-        for (int tile = pair_id; ok && tile < g.num_tiles; tile += num_pairs) {
-            int pm, n;
-            tile_coords(tile, g, pm, n);
-            for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &g_device_error)) { ok = false; break; }
-                if (lane == 0) {
-                    const uint32_t fb_local = smem_u32(&full[stage]);
-                    const uint32_t fb = map_to_rank(fb_local, 0);
-                    if (leader) mbar_arrive_expect_tx(fb_local, PAIR_STAGE_BYTES);
+        if (lane == 0) {  // one lane runs the ring
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_parity = 0;  // per stage: loads issued; parity of the phase they complete
+            bool ok = true;
+            const uint32_t fb0 = map_to_rank(smem_u32(&full[0]), 0);  // the even CTA's stage barriers
+            for (int tile = pair_id; ok && tile < g.num_tiles; tile += num_pairs) {
+                int pm, n;
+                tile_coords(tile, g, pm, n);
+                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                    if (!mbar_wait_fast(smem_u32(&empty[stage]), phase ^ 1u, &g_device_error)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(smem_u32(&full[stage]), PAIR_STAGE_BYTES);
+                    const uint32_t fb = fb0 + (uint32_t)stage * 8u;
                     uint8_t *sa = smem + stage * STAGE_BYTES;
                     tma_load_2d_pair(smem_u32(sa), &tmap_x, kb * BK, pm * 2 * BM + (int)rank * BM, fb);
                     tma_load_2d_pair(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, n * BN + (int)rank * BN_CTA, fb);
+                    armed |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                armed |= 1u << stage;
-                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
+            // The even CTA tracks every copy of the pair on its own stage
+            // barriers: before exiting it waits (bounded) for the last phase
+            // it armed on each stage, so no copy of either CTA is still in
+            // flight (immediate on the normal path, where the MMA consumed
+            // them all).  The odd CTA stays resident until then (cluster
+            // barrier below).
+            if (leader)
+                for (int s2 = 0; s2 < STAGES; ++s2)
+                    if (armed & (1u << s2))
+                        mbar_wait(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, &g_device_error);
         }
-        // The even CTA tracks every copy of the pair on its own stage
-        // barriers: before exiting it waits (bounded) for the last phase it
-        // armed on each stage, so no copy of either CTA is still in flight
-        // (immediate on the normal path, where the MMA consumed them all).
-        // The odd CTA stays resident until then (cluster barrier below).
-        if (leader && lane == 0)
-            for (int s2 = 0; s2 < STAGES; ++s2)
-                if (armed & (1u << s2)) mbar_wait(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, &g_device_error);
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer (even CTA)
-        if (leader) {
+        if (leader && lane == 0) {  // one lane waits and issues
             const uint32_t peer_empty0 = map_to_rank(smem_u32(&empty[0]), 1);
             const uint32_t peer_acc_full0 = map_to_rank(smem_u32(&acc_full[0]), 1);
+            const uint64_t a_desc0 = gemm::sw128_kmajor_desc(smem_u32(smem));  // stage 0; stages move the address field
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -184,36 +187,28 @@ flashnorm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __g
                 gemm::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
                 for (int kb = 0; kb < g.k_blocks; ++kb) {
-                    if (!mbar_wait(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
+                    if (!mbar_wait_fast(smem_u32(&full[stage]), phase, &g_device_error)) { ok = false; break; }
                     gemm::tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
-                        const uint32_t b0 = a0 + A_BYTES;
+                    const uint64_t ad = a_desc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
+                    const uint64_t bd = ad + (uint64_t)(A_BYTES >> 4);
 #pragma unroll
-                        for (int k = 0; k < BK / gemm::UMMA_K; ++k)
-                            umma_pair(d_tmem, gemm::sw128_kmajor_desc(a0 + k * 32),
-                                      gemm::sw128_kmajor_desc(b0 + k * 32), (kb | k) != 0 ? 1u : 0u);
-                        // the stage is free in both CTAs once these MMAs have read it
-                        umma_commit_pair(smem_u32(&empty[stage]));
-                        umma_commit_pair(peer_empty0 + (uint32_t)stage * 8u);
-                    }
-                    __syncwarp();
+                    for (int k = 0; k < BK / gemm::UMMA_K; ++k)
+                        umma_pair(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), (kb | k) != 0 ? 1u : 0u);
+                    // the stage is free in both CTAs once these MMAs have read it
+                    umma_commit_pair(smem_u32(&empty[stage]));
+                    umma_commit_pair(peer_empty0 + (uint32_t)stage * 8u);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                if (lane == 0) {  // both CTAs' accumulators of this tile are complete
-                    umma_commit_pair(smem_u32(&acc_full[acc]));
-                    umma_commit_pair(peer_acc_full0 + (uint32_t)acc * 8u);
-                }
-                __syncwarp();
+                // both CTAs' accumulators of this tile are complete
+                umma_commit_pair(smem_u32(&acc_full[acc]));
+                umma_commit_pair(peer_acc_full0 + (uint32_t)acc * 8u);
             }
             // tensor memory is released only after every MMA issued here has completed
-            if (lane == 0) {
-                umma_commit_pair(smem_u32(drained));
-                mbar_wait(smem_u32(drained), 0u, &g_device_error);
-            }
-            __syncwarp();
+            umma_commit_pair(smem_u32(drained));
+            mbar_wait(smem_u32(drained), 0u, &g_device_error);
         }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2..5, both CTAs)
         // Launched right behind the statistics pass (programmatic dependent

@@ -65,6 +65,14 @@ __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, int
     }
 }
 
+// mbar_wait with the first check inlined: the common case on a pipeline
+// that keeps up (the phase has already completed) costs no call.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, int *err,
+                                               uint64_t timeout_ns = kWaitTimeoutNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait(bar, parity, err, timeout_ns);
+}
+
 // 1-D bulk copy global -> shared, completing `bytes` transactions on `bar`.
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {

@@ -2,8 +2,9 @@
 
 ``QKN_GEMM_KERNEL`` selects the kernel that serves flashnorm_proj calls with a
 given or separately computed 1/rms (and qkv_norm_proj's unscaled projection):
-``pair`` (two CTAs of a cluster per 256 x 256 tile, tcgen05.mma.cta_group::2)
-or ``single`` (one CTA per 128 x 256 tile).  Both accumulate every output in
+the default ``pair`` (two CTAs of a cluster per 256 x 256 tile,
+tcgen05.mma.cta_group::2) or ``single`` (one CTA per 128 x 256 tile, also the
+kernel of the in-kernel statistics form).  Both accumulate every output in
 the same k order in fp32 and scale and round it the same way, so their
 outputs must agree bit for bit; each is also checked against the fp64 oracle
 (relative Frobenius error <= 1e-2 with the original w and W) on shapes with

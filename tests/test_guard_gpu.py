@@ -13,8 +13,8 @@ One case per kernel family: the staged kernel (generic, narrow and
 many-segment flavours), the register kernel (streaming and one-shot), the
 cluster kernel, the element-wise kernel, the partial statistics, the apply
 step of tensor-parallel QK-Norm, the fold (both layouts), the row statistic,
-the projection GEMM (given, separate and in-kernel 1/rms; K-major and
-row-major W'), the fused QKV + QK-Norm GEMM, the RMSNorm-elimination form,
+the projection GEMMs (CTA pair and single CTA; given, separate and
+in-kernel 1/rms; K-major and row-major W'), the fused QKV + QK-Norm GEMM, the RMSNorm-elimination form,
 the no-allocation projection, and the host-buffer pipeline.
 """
 from __future__ import annotations
@@ -162,8 +162,12 @@ def test_inv_rms_stays_inside_output(cuda_lib):
 PROJ_SHAPE = (300, 520, 776)
 
 
+@pytest.mark.parametrize("gemm_kernel", ["pair", "single"])
 @pytest.mark.parametrize("mode", ["separate stats", "in-kernel stats", "given inv_rms", "row-major W'"])
-def test_projection_stays_inside_output(cuda_lib, mode):
+def test_projection_stays_inside_output(cuda_lib, mode, gemm_kernel, monkeypatch):
+    # the CTA-pair kernel (default) and the single-CTA kernel; the in-kernel
+    # statistics form always runs on the single-CTA kernel
+    monkeypatch.setenv("QKN_GEMM_KERNEL", gemm_kernel)
     M, K, N = PROJ_SHAPE
     inp = W.make_flashnorm_inputs(seed=5, M=M, K=K, N=N)
     x = inp["x"].to(DEV)

@@ -18,6 +18,7 @@
 #include <string.h>
 
 #include "gemm_tc.cuh"
+#include "pair_tc.cuh"
 #include "qkn_common.cuh"
 #include "qkn_sync.cuh"
 

@@ -29,32 +29,9 @@
 // and each producer for all the copies it issued.
 #pragma once
 
+// (pair_tc.cuh, the tile shape and helpers, is included at file scope by flashnorm.cu)
+
 namespace pair {
-
-constexpr int BM = 128;                            // x rows per CTA (256 per pair)
-constexpr int BN = 256;                            // columns per pair tile
-constexpr int BN_CTA = 128;                        // W' rows loaded by each CTA
-constexpr int BK = 64;                             // bf16: one 128-byte swizzle row
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK * 2;               // 16 KiB
-constexpr int B_BYTES = BN_CTA * BK * 2;           // 16 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 32 KiB per CTA
-constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;  // bytes completing on the even CTA's barrier
-constexpr int ACC_COLS = BN;
-constexpr int TMEM_COLS = 2 * ACC_COLS;            // double-buffered accumulator
-constexpr int THREADS = 192;
-constexpr int EPI_BYTES = 4 * 2 * 2048;            // two 32 x 32 bf16 staging tiles per epilogue warp
-constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;  // + 1 KiB for alignment
-constexpr int GROUP_M = 8;                         // pair row blocks (256 rows) per raster group
-
-static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-
-// kind::f16 instruction descriptor: bf16 A and B (both K-major), fp32 D,
-// M = 256 (the pair), N = 256.
-constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                ((uint32_t)(2 * BM >> 4) << 24);
 
 struct Args {
     const float *inv_rms;  // [M] 1/rms per row (unit_scale == 0)
@@ -73,28 +50,6 @@ __device__ __forceinline__ void tile_coords(int tile, const Args &g, int &pm, in
     const int in_group = tile - group * group_tiles;
     pm = first + in_group % rows_in_group;
     n = in_group / rows_in_group;
-}
-
-// 2-D tensor copy into this CTA's shared memory whose bytes complete on the
-// barrier at shared::cluster address `bar` (the even CTA's).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kInstrDesc), "r"(accumulate));
-}
-
-// Arrives on the barrier at shared::cluster address `bar` once every MMA
-// this thread issued so far has completed.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(bar) : "memory");
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)

@@ -158,6 +158,108 @@ __device__ __forceinline__ void load_w8(const void *w, int w_f32, int c, float (
     }
 }
 
+// The epilogue of one accumulator tile for the 32 rows of this warp (TMEM
+// lane quarter `quarter` of the tile's 128-row block `mb`): QK-Norm's tile
+// partials published and exchanged for q and k tiles, then the scaled tile
+// stored in bf16.  `skip` (testing only) leaves this warp's arrival out.
+__device__ __forceinline__ void epilogue_tile(const Args &g, const CUtensorMap *tmap_y, int mb, const Tile &t,
+                                              uint32_t acc_tmem, uint32_t epi, int &issued, int quarter, int lane,
+                                              bool skip) {
+    const int lrow = quarter * 32 + lane;
+    const int row = mb * BM + lrow;
+    const bool row_ok = row < g.M;
+    const float r = g.inv_rms == nullptr ? 1.f : (row_ok ? __ldg(g.inv_rms + row) : 0.f);
+    const uint32_t tbase = acc_tmem + ((uint32_t)(quarter * 32) << 16);
+    const int ncols = min(BN, t.col_end - t.col0);  // columns of this tile inside its section
+    const int nchunks = (ncols + 31) / 32;
+    float inv_qk = 1.f;
+    const void *w = nullptr;
+    int w0 = 0;
+    if (t.sec < 2) {
+        // pass 1: this tile's share of the row's sum of squares of u = r * acc
+        float2 ss = make_float2(0.f, 0.f);
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            gemm::tmem_ld_32cols(tbase + c * 32, v);
+            const int valid = ncols - c * 32;  // a multiple of 8
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                if (j < valid) {
+                    const float2 u = make_float2(__uint_as_float(v[j]) * r, __uint_as_float(v[j + 1]) * r);
+                    ss = __ffma2_rn(u, u, ss);
+                }
+            }
+        }
+        float *prow = g.partial + ((size_t)t.sec * g.m_blocks * BM + (size_t)row) * g.pstride;
+        prow[t.n] = ss.x + ss.y;
+        __threadfence();
+        __syncwarp();
+        unsigned *cnt = g.count + (mb * 2 + t.sec) * 4 + quarter;
+        if (lane == 0 && !skip) red_release_add(cnt, 1u);
+        const int ntiles = t.sec == 0 ? g.tq : g.tk;
+        if (!wait_count(cnt, (unsigned)ntiles, g.wait_ns) && lane == 0) atomicExch(&g_qkv_error, 1);
+        // fixed-order combine of the row's per-tile partial sums
+        float S = 0.f;
+        for (int i = 0; i < ntiles; ++i) S += __ldcg(prow + i);
+        const int d = t.sec == 0 ? g.nq : g.nk;
+        inv_qk = rsqrtf(S / (float)d + g.eps);
+        w = t.sec == 0 ? g.wq : g.wk;
+        w0 = t.col0 - (t.sec == 0 ? 0 : g.nq);
+    }
+    // pass 2: y = ((r * acc) * inv_qk) * w for q and k, r * acc for v; bf16 out
+    const int row0 = mb * BM + quarter * 32;
+    __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+        uint32_t v[32];
+        gemm::tmem_ld_32cols(tbase + c * 32, v);
+        const int base = c * 32;
+        const bool whole = base + 32 <= ncols;  // the same for the whole warp
+        const uint32_t buf = epi + (uint32_t)(issued & 1) * 2048u;
+        if (whole) {
+            if (lane == 0 && issued >= 2) bulk_wait_read1();  // the store two blocks back has read it
+            __syncwarp();
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int off = base + j * 8;
+            if (whole || (row_ok && off < ncols)) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * j + e]) * r;
+                if (t.sec < 2) {
+                    float wv[8];
+                    load_w8(w, g.w_f32, w0 + off, wv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = (f[e] * inv_qk) * wv[e];
+                }
+                uint4 o;
+                o.x = pack_bf16x2(f[0], f[1]);
+                o.y = pack_bf16x2(f[2], f[3]);
+                o.z = pack_bf16x2(f[4], f[5]);
+                o.w = pack_bf16x2(f[6], f[7]);
+                if (whole) {
+                    const uint32_t dst = buf + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                 ::"r"(dst), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w) : "memory");
+                } else {
+                    *reinterpret_cast<uint4 *>(yrow + t.col0 + off) = o;
+                }
+            }
+        }
+        if (whole) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (row0 < g.M) tma_store_2d(tmap_y, buf, t.col0 + base, row0);
+                bulk_commit();
+            }
+            ++issued;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_y, const Args g) {
@@ -195,69 +297,66 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t armed = 0, armed_parity = 0;  // per stage: loads issued; parity of the phase they complete
-        bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
-            const Tile t = tile_of(tile, g);
-            for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, &g_qkv_error, g.wait_ns)) { ok = false; break; }
-                if (lane == 0) {
+        if (lane == 0) {  // one lane runs the ring
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_parity = 0;  // per stage: loads issued; parity of the phase they complete
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x) {
+                const Tile t = tile_of(tile, g);
+                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                    if (!mbar_wait_fast(smem_u32(&empty[stage]), phase ^ 1u, &g_qkv_error, g.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
                     const uint32_t fb = smem_u32(&full[stage]);
                     uint8_t *sa = smem + stage * STAGE_BYTES;
                     mbar_arrive_expect_tx(fb, STAGE_BYTES);
                     tma_load_2d(smem_u32(sa), &tmap_x, kb * BK, t.m_blk * BM, fb);
                     tma_load_2d(smem_u32(sa + A_BYTES), &tmap_w, kb * BK, t.col0, fb);
+                    armed |= 1u << stage;
+                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                armed |= 1u << stage;
-                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-        }
-        // No copy may still be writing shared memory when the CTA exits: wait
-        // (bounded) for the last phase armed on every stage (immediate on the
-        // normal path, where the MMA warp consumed them all).
-        if (lane == 0)
+            // No copy may still be writing shared memory when the CTA exits:
+            // wait (bounded) for the last phase armed on every stage
+            // (immediate on the normal path, where the MMA warp consumed them all).
             for (int s2 = 0; s2 < STAGES; ++s2)
                 if (armed & (1u << s2))
                     mbar_wait(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, &g_qkv_error, g.wait_ns);
+        }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
-        int stage = 0;
-        uint32_t phase = 0;
-        int it = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x, ++it) {
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, &g_qkv_error, g.wait_ns)) break;
-            gemm::tc_fence_after();
-            const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-            for (int kb = 0; kb < g.k_blocks; ++kb) {
-                if (!mbar_wait(smem_u32(&full[stage]), phase, &g_qkv_error, g.wait_ns)) { ok = false; break; }
+        if (lane == 0) {  // one lane waits and issues; stages move the descriptors' address field
+            const uint64_t a_desc0 = gemm::sw128_kmajor_desc(smem_u32(smem));
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait_fast(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, &g_qkv_error, g.wait_ns)) break;
                 gemm::tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t b0 = a0 + A_BYTES;
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < g.k_blocks; ++kb) {
+                    if (!mbar_wait_fast(smem_u32(&full[stage]), phase, &g_qkv_error, g.wait_ns)) { ok = false; break; }
+                    gemm::tc_fence_after();
+                    const uint64_t ad = a_desc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
+                    const uint64_t bd = ad + (uint64_t)(A_BYTES >> 4);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k)
-                        gemm::umma_bf16(d_tmem, gemm::sw128_kmajor_desc(a0 + k * 32),
-                                        gemm::sw128_kmajor_desc(b0 + k * 32), (kb | k) != 0 ? 1u : 0u);
+                        gemm::umma_bf16(d_tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), (kb | k) != 0 ? 1u : 0u);
                     gemm::umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                if (!ok) break;
+                gemm::umma_commit(smem_u32(&acc_full[acc]));
             }
-            if (!ok) break;
-            if (lane == 0) gemm::umma_commit(smem_u32(&acc_full[acc]));
-            __syncwarp();
-        }
-        // Tensor memory is released only after every MMA issued here has
-        // completed, also when a wait above gave up with MMAs in flight.
-        if (lane == 0) {
+            // Tensor memory is released only after every MMA issued here has
+            // completed, also when a wait above gave up with MMAs in flight.
             gemm::umma_commit(smem_u32(drained));
             mbar_wait(smem_u32(drained), 0u, &g_qkv_error, g.wait_ns);
         }
@@ -265,7 +364,6 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
         const int quarter = warp & 3;  // TMEM lanes 32 * quarter ... of the accumulator
-        const int lrow = quarter * 32 + lane;
         // 32 x 32 output blocks go out through shared memory and one TMA store
         // each (two alternating staging buffers per warp, 64-byte swizzle); a
         // block that a section ends inside is stored lane by lane instead
@@ -278,99 +376,8 @@ qkv_qknorm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             const uint32_t acc_phase = (it >> 1) & 1;
             if (!mbar_wait(smem_u32(&acc_full[acc]), acc_phase, &g_qkv_error, g.wait_ns)) break;
             gemm::tc_fence_after();
-            const int row = t.m_blk * BM + lrow;
-            const bool row_ok = row < g.M;
-            const float r = g.inv_rms == nullptr ? 1.f : (row_ok ? __ldg(g.inv_rms + row) : 0.f);
-            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
-            const int ncols = min(BN, t.col_end - t.col0);  // columns of this tile inside its section
-            const int nchunks = (ncols + 31) / 32;
-            float inv_qk = 1.f;
-            const void *w = nullptr;
-            int w0 = 0;
-            if (t.sec < 2) {
-                // pass 1: this tile's share of the row's sum of squares of u = r * acc
-                float2 ss = make_float2(0.f, 0.f);
-#pragma unroll 1
-                for (int c = 0; c < nchunks; ++c) {
-                    uint32_t v[32];
-                    gemm::tmem_ld_32cols(tbase + c * 32, v);
-                    const int valid = ncols - c * 32;  // a multiple of 8
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        if (j < valid) {
-                            const float2 u = make_float2(__uint_as_float(v[j]) * r, __uint_as_float(v[j + 1]) * r);
-                            ss = __ffma2_rn(u, u, ss);
-                        }
-                    }
-                }
-                float *prow = g.partial + ((size_t)t.sec * g.m_blocks * BM + (size_t)row) * g.pstride;
-                prow[t.n] = ss.x + ss.y;
-                __threadfence();
-                __syncwarp();
-                unsigned *cnt = g.count + (t.m_blk * 2 + t.sec) * 4 + quarter;
-                const bool skip = g.skip_arrival && blockIdx.x == 0 && it == 0 && quarter == 0;
-                if (lane == 0 && !skip) red_release_add(cnt, 1u);
-                const int ntiles = t.sec == 0 ? g.tq : g.tk;
-                if (!wait_count(cnt, (unsigned)ntiles, g.wait_ns) && lane == 0) atomicExch(&g_qkv_error, 1);
-                // fixed-order combine of the row's per-tile partial sums
-                float S = 0.f;
-                for (int i = 0; i < ntiles; ++i) S += __ldcg(prow + i);
-                const int d = t.sec == 0 ? g.nq : g.nk;
-                inv_qk = rsqrtf(S / (float)d + g.eps);
-                w = t.sec == 0 ? g.wq : g.wk;
-                w0 = t.col0 - (t.sec == 0 ? 0 : g.nq);
-            }
-            // pass 2: y = ((r * acc) * inv_qk) * w for q and k, r * acc for v; bf16 out
-            const int row0 = t.m_blk * BM + quarter * 32;
-            __nv_bfloat16 *yrow = g.y + (int64_t)(row_ok ? row : 0) * g.N;
-#pragma unroll 1
-            for (int c = 0; c < nchunks; ++c) {
-                uint32_t v[32];
-                gemm::tmem_ld_32cols(tbase + c * 32, v);
-                const int base = c * 32;
-                const bool whole = base + 32 <= ncols;  // the same for the whole warp
-                const uint32_t buf = epi + (uint32_t)(issued & 1) * 2048u;
-                if (whole) {
-                    if (lane == 0 && issued >= 2) bulk_wait_read1();  // the store two blocks back has read it
-                    __syncwarp();
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int off = base + j * 8;
-                    if (whole || (row_ok && off < ncols)) {
-                        float f[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * j + e]) * r;
-                        if (t.sec < 2) {
-                            float wv[8];
-                            load_w8(w, g.w_f32, w0 + off, wv);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) f[e] = (f[e] * inv_qk) * wv[e];
-                        }
-                        uint4 o;
-                        o.x = pack_bf16x2(f[0], f[1]);
-                        o.y = pack_bf16x2(f[2], f[3]);
-                        o.z = pack_bf16x2(f[4], f[5]);
-                        o.w = pack_bf16x2(f[6], f[7]);
-                        if (whole) {
-                            const uint32_t dst = buf + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16);
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                         ::"r"(dst), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w) : "memory");
-                        } else {
-                            *reinterpret_cast<uint4 *>(yrow + t.col0 + off) = o;
-                        }
-                    }
-                }
-                if (whole) {
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (row0 < g.M) tma_store_2d(&tmap_y, buf, t.col0 + base, row0);
-                        bulk_commit();
-                    }
-                    ++issued;
-                }
-            }
+            epilogue_tile(g, &tmap_y, t.m_blk, t, tmem_base + acc * ACC_COLS, epi, issued, quarter, lane,
+                          g.skip_arrival && blockIdx.x == 0 && it == 0 && quarter == 0);
             gemm::tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));

@@ -687,7 +687,8 @@ def host_pipeline(hx, hy, call, dev, nchunks=8):
     return step
 
 
-FN_SRC = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
+FN_SRC = ["rmsnorm_qknorm_b200/csrc/flashnorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_pair.cuh",
+          "rmsnorm_qknorm_b200/csrc/pair_tc.cuh", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
           "rmsnorm_qknorm_b200/csrc/qkn_common.cuh", "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
 QKV_SRC = ["rmsnorm_qknorm_b200/csrc/qkv_qknorm.cu", "rmsnorm_qknorm_b200/csrc/gemm_tc.cuh",
            "rmsnorm_qknorm_b200/csrc/qkn_common.cuh", "rmsnorm_qknorm_b200/csrc/qkn_sync.cuh"]
@@ -789,7 +790,11 @@ def projection_roofline(kind, avg_gemm_ms, clk, src):
     wl = W.FLASHNORM_WORKLOAD
     pk, pk_kind = peaks()
     tflops = wl.flops() / (avg_gemm_ms * 1e-3) / 1e12
-    kernel = "flashnorm_gemm_kernel" if kind == "flashnorm_proj" else "qkv_qknorm_gemm_kernel"
+    if kind == "flashnorm_proj":  # the CTA-pair kernel unless the single-CTA one was selected
+        kernel = ("flashnorm_gemm_kernel" if os.environ.get("QKN_GEMM_KERNEL") == "single"
+                  else "flashnorm_gemm_pair_kernel")
+    else:
+        kernel = "qkv_qknorm_gemm_kernel"
     # algorithmic bytes of one launch: x and W' read once, y written once
     algo = (wl.M * wl.K + wl.N * wl.K + wl.M * wl.N) * 2
     t = traffic_for(kernel, kind, src, algo)

@@ -78,6 +78,26 @@ def test_noalloc_matches_allocating_entry_point():
     assert lib.qkn_check_device(None) == 0, lib.qkn_last_error()
 
 
+def test_noalloc_at_the_row_limit():
+    # exactly as many rows as the fixed scratch holds: every entry of it is written
+    # and read, and the result is still the allocating entry point's, bit for bit
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test collected on a machine without CUDA")
+    lib, f = _noalloc_fn()
+    M, K, N = MAX_ROWS, 64, 72
+    inp = W.make_flashnorm_inputs(seed=9, M=16, K=K, N=N)  # weights; rows drawn below
+    g = torch.Generator().manual_seed(10)
+    x = (torch.randn(M, K, generator=g) * torch.exp(torch.randn(M, 1, generator=g))).to(torch.bfloat16).to(DEV)
+    Wf = qk.flashnorm_fold_weights(inp["w"].to(DEV), inp["W"].to(DEV))
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    st = f(x.data_ptr(), Wf.data_ptr(), y.data_ptr(), M, N, K, 1, inp["eps"], torch.cuda.current_stream().cuda_stream)
+    assert st == 0, lib.qkn_last_error().decode()
+    y_ref = qk.flashnorm_proj(x, Wf, inp["eps"])
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    assert lib.qkn_check_device(None) == 0, lib.qkn_last_error()
+
+
 def test_noalloc_rejects_rows_beyond_the_fixed_scratch():
     lib, f = _noalloc_fn()
     # validated on the host before anything is launched: pointers are never touched

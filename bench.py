@@ -579,14 +579,17 @@ def run_qknorm(args, rank, world, local, pg):
     # The other graded workloads, measured after the headline on the same GPU,
     # each with its own clock record: the prefill GQA QK-Norm (HBM roofline)
     # and the two tensor-core projections (bf16 peak).
+    # At N > 1 those per-GPU figures are the N = 1 line's; the line carries
+    # the tensor-parallel comparison across the ranks instead.
     extras = {}
     if args.workload == QK_DEFAULT and args.tokens is None and not args.no_extras:
-        extras["prefill_gqa"] = extra_qknorm("prefill_gqa", dev, local, pg, rank)
-        torch.cuda.empty_cache()
-        for kind in ("flashnorm_proj", "qkv_proj_qknorm"):
-            extras[kind] = extra_projection(kind, dev, local, pg, rank)
+        if world == 1:
+            extras["prefill_gqa"] = extra_qknorm("prefill_gqa", dev, local, pg, rank)
             torch.cuda.empty_cache()
-        if world > 1:
+            for kind in ("flashnorm_proj", "qkv_proj_qknorm"):
+                extras[kind] = extra_projection(kind, dev, local, pg, rank)
+                torch.cuda.empty_cache()
+        else:
             # tensor-parallel QK-Norm of the prefill GQA layer split over all
             # the ranks (S = world): SwiftQK's scalar exchange against the
             # All-Gather form, over the real interconnect

@@ -58,6 +58,71 @@ __device__ __forceinline__ RowJob pick_job(const RowArgs &a, int which) {
     return J;
 }
 
+// Per-segment sums of squares of a thread's chunks v[i] (chunk i * tpr + t
+// of its row): each chunk's sum s (a fused multiply-add chain over its
+// elements from zero) is added into acc[(i * tpr + t) / seg_chunks], each
+// accumulator taking its chunks in increasing i.  When a segment is q whole
+// chunk slots (seg_chunks = q * tpr), slot i lies in segment i / q for every
+// thread, so q = 1, 2, 4 and q >= CPT (then the row is one segment: its
+// chunks fill at most tpr * CPT slots) add each sum straight into its
+// accumulator; other widths compute the segment index per chunk and add
+// the sum to every accumulator, zero to all but the chunk's own.  Adding zero
+// leaves a non-negative sum's bits unchanged, so both forms give the same
+// bits.  SLOTS = false compiles the per-chunk form alone: the normalising
+// kernels keep it (measured on B200: the streaming kernel ran 4-17 % slower
+// with both forms compiled in, while the statistics alone, bound by issue
+// slots, ran 17-24 % faster with the slot form).
+template <typename TA, int CPT, bool SLOTS>
+__device__ __forceinline__ void segment_sums(const uint4 (&v)[CPT], int t, int tpr, const RowJob &J,
+                                             float (&acc)[kFastMaxSeg]) {
+    static_assert(CPT == kFastMaxSeg, "slot i's segment is i / q < CPT");
+    constexpr int E = Chunk<TA>::E;
+#pragma unroll
+    for (int j = 0; j < kFastMaxSeg; ++j) acc[j] = 0.f;
+    const int q = (J.seg_chunks & (tpr - 1)) == 0 ? J.seg_chunks >> J.tpr_log2 : 0;
+    if (SLOTS && (q == 1 || q == 2 || q == 4 || q >= CPT)) {
+        float sq[CPT];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            float f[E];
+            Chunk<TA>::unpack(v[i], f);
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+            sq[i] = s;
+        }
+        if (q == 1) {
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) acc[i] += sq[i];
+        } else if (q == 2) {
+#pragma unroll
+            for (int j = 0; j < CPT / 2; ++j) acc[j] = (acc[j] + sq[2 * j]) + sq[2 * j + 1];
+        } else if (q == 4) {
+#pragma unroll
+            for (int j = 0; j < CPT / 4; ++j)
+                acc[j] = (((acc[j] + sq[4 * j]) + sq[4 * j + 1]) + sq[4 * j + 2]) + sq[4 * j + 3];
+        } else {
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) acc[0] += sq[i];
+        }
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * tpr + t;
+        float f[E];
+        Chunk<TA>::unpack(v[i], f);
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
+        // floor(c / seg_chunks): (c + 0.5) / seg_chunks is never an integer, and
+        // the fp32 error stays below 0.5 / seg_chunks for c < 2^22 (host-checked)
+        const int seg = __float2int_rz(((float)c + 0.5f) * J.inv_seg_chunks);
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j) acc[j] += (j == seg) ? s : 0.f;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Vectorised kernel: a row lives in the registers of 2^tpr_log2 threads, each
 // holding up to CPT 16-byte chunks (chunk c of the row sits in thread c % tpr,
@@ -94,22 +159,7 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) rownorm_vec_kernel(const 
 
     // 2. per-thread partial sum of squares of each segment
     float acc[kFastMaxSeg];
-#pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) acc[j] = 0.f;
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int c = i * tpr + t;
-        float f[E];
-        Chunk<TA>::unpack(v[i], f);
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
-        // floor(c / seg_chunks): (c + 0.5) / seg_chunks is never an integer, and
-        // the fp32 error stays below 0.5 / seg_chunks for c < 2^22 (host-checked)
-        const int seg = __float2int_rz(((float)c + 0.5f) * J.inv_seg_chunks);
-#pragma unroll
-        for (int j = 0; j < kFastMaxSeg; ++j) acc[j] += (j == seg) ? s : 0.f;
-    }
+    segment_sums<TA, CPT, STATS>(v, t, tpr, J, acc);
 
     // 3. reduce each segment over the threads of the row (fixed tree)
     const int n_seg = a.n_seg;
@@ -300,20 +350,7 @@ __device__ __forceinline__ void process_group(const RowArgs &a, int64_t g, int64
     const int nchunks = J.nchunks;
 
     float acc[kFastMaxSeg];
-#pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) acc[j] = 0.f;
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int c = i * tpr + t;
-        float f[E];
-        Chunk<TA>::unpack(v[i], f);
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) s = fmaf(f[e], f[e], s);
-        const int seg = __float2int_rz(((float)c + 0.5f) * J.inv_seg_chunks);
-#pragma unroll
-        for (int j = 0; j < kFastMaxSeg; ++j) acc[j] += (j == seg) ? s : 0.f;
-    }
+    segment_sums<TA, CPT, false>(v, t, tpr, J, acc);
     const int n_seg = a.n_seg;
 #pragma unroll
     for (int j = 0; j < kFastMaxSeg; ++j) {

@@ -324,6 +324,37 @@ def test_many_segments_staged(cuda_lib, dtype, dq, dk, n_seg):
     assert_f32_close(p, oracle.segment_partials(q.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials n_seg={n_seg}")
 
 
+@pytest.mark.parametrize("T,d,pad,n_seg,dtype", [
+    (20001, 1024, 0, 8, torch.bfloat16),    # a segment is one chunk slot of each thread
+    (20001, 1024, 40, 4, torch.bfloat16),   # two slots; pitched rows
+    (200001, 128, 0, 1, torch.bfloat16),    # one segment: the whole row
+    (40001, 64, 8, 2, torch.bfloat16),      # one chunk per row (one thread), pitched
+    (30001, 1024, 0, 8, torch.float32),     # 4 KiB fp32 rows: 32 threads per row
+    (30001, 2048, 0, 2, torch.bfloat16),    # four slots
+    (20001, 640, 0, 8, torch.bfloat16),     # segments of 10 chunks over 16 threads: per-chunk index
+    (60001, 512, 8, 16, torch.bfloat16),    # many segments, pitched
+    (10001, 2048, 0, 64, torch.bfloat16),   # many segments, 4 KiB rows
+])
+def test_partial_stats_narrow_rows(cuda_lib, T, d, pad, n_seg, dtype):
+    # the statistics alone of rows up to 4 KiB (the one-shot register kernel, and
+    # for more than 8 segments the streaming one; segments of 1, 2 or 4 chunk slots
+    # per thread, whole rows, and other widths): many row groups, a ragged last
+    # one, pitched rows; the partials are the ones qknorm_fused combines for the
+    # same rows (its output is reproduced bit for bit from them) and match the oracle
+    g = torch.Generator().manual_seed(T + d + n_seg)
+    x_full = (torch.randn(T, d + pad, generator=g) * 2).to(dtype).to(DEV)
+    x = x_full[:, :d]
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(dtype).to(DEV)
+    p = qk.rmsnorm_partial_stats(x, n_seg)
+    y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, n_seg)
+    y2 = qk.rmsnorm_apply_partials(x, w, p, d, 1e-6)
+    torch.cuda.synchronize()
+    bits = (lambda t: t.view(torch.int16)) if dtype == torch.bfloat16 else (lambda t: t.view(torch.int32))
+    assert torch.equal(bits(y2), bits(y))
+    assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL,
+                     what=f"partials T={T} d={d} n_seg={n_seg}")
+
+
 @pytest.mark.parametrize("T,dq,dk", [(50001, 128, 128), (20001, 1024, 1024), (10001, 2048, 512)])
 def test_register_stream_many_groups(cuda_lib, T, dq, dk):
     # enough rows that each persistent block of the streaming register kernel walks

@@ -273,11 +273,16 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
         J.w_offset = a.w_bytes;
         if (!STATS) a.w_bytes += (int)(t.d * 4);
         J.rows_per_tile = stage_bytes / J.row_bytes;
-        // narrow rows of 32, 64 or 128 chunks whose segments are whole power-of-two lane groups
-        J.narrow_cpl = 0;
-        if (n_seg <= kFastMaxSeg && J.nchunks % 32 == 0 && J.nchunks <= 128) {
-            const int cpl = J.nchunks / 32, lps = 32 / n_seg;
-            if (lps * n_seg == 32 && (lps & (lps - 1)) == 0 && J.seg_chunks == cpl * lps) J.narrow_cpl = cpl;
+        // rows the register kernels take on their own keep those kernels'
+        // arithmetic (staged::process_rows_reg), a whole number of warp
+        // passes per tile (a stage holds at least one: 32 / tpr rows of at
+        // most tpr x 128 bytes)
+        J.reg_tpr_log2 = -1;
+        J.inv_seg_chunks = 1.0f / (float)J.seg_chunks;
+        if (n_seg <= kFastMaxSeg && J.nchunks <= 32 * stream::CPT) {
+            J.reg_tpr_log2 = ceil_log2((J.nchunks + stream::CPT - 1) / stream::CPT);
+            const int rpw = 32 >> J.reg_tpr_log2;
+            if (J.rows_per_tile >= rpw) J.rows_per_tile = J.rows_per_tile / rpw * rpw;
         }
         J.ntiles = (rows + J.rows_per_tile - 1) / J.rows_per_tile;
         a.total_tiles += J.ntiles;
@@ -286,9 +291,9 @@ qkn_status launch_staged(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, 
     const int64_t grid = a.total_tiles < sm_count() ? a.total_tiles : sm_count();
     if (n_seg > kFastMaxSeg)
         return launch_staged_kernel<TA, TW, STATS, staged::kFlavorManySeg>(a, (int)grid, smem, s);
-    bool narrow = false;
-    for (int i = 0; i < njobs; ++i) narrow = narrow || a.job[i].narrow_cpl != 0;
-    if (narrow) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorNarrow>(a, (int)grid, smem, s);
+    bool reg_rows = false;
+    for (int i = 0; i < njobs; ++i) reg_rows = reg_rows || a.job[i].reg_tpr_log2 >= 0;
+    if (reg_rows) return launch_staged_kernel<TA, TW, STATS, staged::kFlavorRegRows>(a, (int)grid, smem, s);
     return launch_staged_kernel<TA, TW, STATS, staged::kFlavorGeneric>(a, (int)grid, smem, s);
 }
 
@@ -334,15 +339,23 @@ qkn_status launch_stats_direct(const Tensor2 &t, int64_t rows, int n_seg, float 
     return check_launch("rowstats_direct_kernel launch");
 }
 
-template <typename TA, typename TW, bool STATS>
-qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps,
-                    float *partial, cudaStream_t s) {
-    constexpr int E = Chunk<TA>::E;
-    RowArgs a{};
-    a.n_seg = n_seg;
-    a.eps = eps;
-    a.partial = partial;
+// The kernel a set of rows takes, and its launch parameters.  The per-row
+// arithmetic of each kind depends on the row's own width, dtype and n_seg
+// (and, for clusters, on the cluster size), never on the rows that share
+// the launch; dispatch keeps it that way for two jobs (below).
+enum class Kernel { kRegisterMany, kStaged, kRegister, kCluster, kScalar };
+struct Route {
+    Kernel kind;
+    int cfg;                 // kRegister: kVecCfgs entry
+    bool stream;             // kRegister: the streaming form
+    int cluster;             // kCluster: CTAs per row
+    int warps, spw, sb;      // kStaged: ring geometry
+};
 
+template <typename TA, typename TW, bool STATS>
+Route plan(const Tensor2 *ts, int njobs, int n_seg) {
+    constexpr int E = Chunk<TA>::E;
+    Route r{};
     // 16-byte rows with whole chunks per segment take the vector paths
     bool chunked = true;
     int64_t max_chunks = 0;
@@ -383,31 +396,27 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
     // with its many-segment statistic (per-chunk sums parked in shared memory,
     // each segment added in chunk order by one lane).
     if (many && max_chunks <= 32 * stream::CPT && max_row_bytes <= kRegisterMaxRowBytes) {
-        setup_vec_jobs<TA>(a, ts, njobs, rows, n_seg, stream::CPT, stream::BLOCK);
-        return launch_vec_stream<TA, TW, STATS, true>(a, njobs, s);
+        r.kind = Kernel::kRegisterMany;
+        return r;
     }
     if ((vec && max_row_bytes > (STATS ? kRegisterMaxRowBytesStats : kRegisterMaxRowBytes)) || many) {
         int64_t w_bytes = 0;
         for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
-        int warps = 0, spw = 0, sb = 0;
-        if (staged_geometry(max_row_bytes, w_bytes, n_seg, &warps, &spw, &sb)) {
-            if (STATS) return launch_stats_direct<TA>(ts[0], rows, n_seg, partial, s);
-            return launch_staged<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, warps, spw, sb, s);
+        if (staged_geometry(max_row_bytes, w_bytes, n_seg, &r.warps, &r.spw, &r.sb)) {
+            r.kind = Kernel::kStaged;
+            return r;
         }
     }
-
     if (vec) {
-        setup_vec_jobs<TA>(a, ts, njobs, rows, n_seg, kVecCfgs[cfg].cpt, kVecCfgs[cfg].block);
+        r.kind = Kernel::kRegister;
+        r.cfg = cfg;
         // narrow rows (at most 32 threads per row) stream through persistent
         // blocks that load the next rows while they normalise the current ones
         // (the statistics alone keep the one-shot form, which measured faster
         // for them than the streaming form and than a ring of bulk copies)
-        if (!STATS && cfg == 0 && max_chunks <= 32 * stream::CPT)
-            return launch_vec_stream<TA, TW, STATS>(a, njobs, s);
-        if (cfg == 0) return launch_vec<TA, TW, 8, 256, STATS>(a, njobs, s);
-        return launch_vec<TA, TW, 8, 1024, STATS>(a, njobs, s);
+        r.stream = !STATS && cfg == 0 && max_chunks <= 32 * stream::CPT;
+        return r;
     }
-
     // chunked rows with more than 8 segments, or wider than one CTA's
     // registers hold: spread each row over the CTAs of a cluster
     if (chunked) {
@@ -415,10 +424,39 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
         if (need <= cl::kMaxCluster) {
             int C = 1;
             while (C < need) C <<= 1;
-            return launch_cluster<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, C, s);
+            r.kind = Kernel::kCluster;
+            r.cluster = C;
+            return r;
         }
     }
+    r.kind = Kernel::kScalar;
+    return r;
+}
 
+template <typename TA, typename TW, bool STATS>
+qkn_status launch_route(const Route &r, const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps,
+                        float *partial, cudaStream_t s) {
+    RowArgs a{};
+    a.n_seg = n_seg;
+    a.eps = eps;
+    a.partial = partial;
+    switch (r.kind) {
+    case Kernel::kRegisterMany:
+        setup_vec_jobs<TA>(a, ts, njobs, rows, n_seg, stream::CPT, stream::BLOCK);
+        return launch_vec_stream<TA, TW, STATS, true>(a, njobs, s);
+    case Kernel::kStaged:
+        if (STATS) return launch_stats_direct<TA>(ts[0], rows, n_seg, partial, s);
+        return launch_staged<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, r.warps, r.spw, r.sb, s);
+    case Kernel::kRegister:
+        setup_vec_jobs<TA>(a, ts, njobs, rows, n_seg, kVecCfgs[r.cfg].cpt, kVecCfgs[r.cfg].block);
+        if (r.stream) return launch_vec_stream<TA, TW, STATS>(a, njobs, s);
+        if (r.cfg == 0) return launch_vec<TA, TW, 8, 256, STATS>(a, njobs, s);
+        return launch_vec<TA, TW, 8, 1024, STATS>(a, njobs, s);
+    case Kernel::kCluster:
+        return launch_cluster<TA, TW, STATS>(ts, njobs, rows, n_seg, eps, partial, r.cluster, s);
+    case Kernel::kScalar:
+        break;
+    }
     for (int i = 0; i < njobs; ++i) {
         const Tensor2 &t = ts[i];
         RowJob &J = a.job[i];
@@ -434,6 +472,34 @@ qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float
     if (blocks > 0x7fffffffLL) return fail(QKN_ERR_SHAPE, "too many rows for one launch");
     rownorm_scalar_kernel<TA, TW, STATS><<<(unsigned)blocks, kScalarBlock, 0, s>>>(a);
     return check_launch("rownorm_scalar_kernel launch");
+}
+
+// q and k share one launch when each would take the same kind of kernel on
+// its own (the same cluster size, for clusters), or when one would take the
+// register kernels and the other the staged kernel with at most 8 segments:
+// the staged kernel then keeps the register kernels' arithmetic for the
+// narrow rows (the prefill arrangement, 5120 + 1024).  Otherwise each goes
+// to its own kernel, one launch after the other on the stream.  So the bits
+// of a row depend on its own tensor's width, dtype, alignment and n_seg
+// only: normalised beside any partner, or alone, it comes out the same, and
+// rmsnorm_partial_stats gives the partial sums it was normalised with.
+template <typename TA, typename TW, bool STATS>
+qkn_status dispatch(const Tensor2 *ts, int njobs, int64_t rows, int n_seg, float eps,
+                    float *partial, cudaStream_t s) {
+    const Route joint = plan<TA, TW, STATS>(ts, njobs, n_seg);
+    if (njobs == 2) {
+        const Route r0 = plan<TA, TW, STATS>(ts, 1, n_seg), r1 = plan<TA, TW, STATS>(ts + 1, 1, n_seg);
+        const bool same = r0.kind == r1.kind && joint.kind == r0.kind &&
+                          (r0.kind != Kernel::kCluster || (r0.cluster == r1.cluster && joint.cluster == r0.cluster));
+        const bool reg_in_staged = joint.kind == Kernel::kStaged && n_seg <= kFastMaxSeg &&
+                                   ((r0.kind == Kernel::kRegister && r1.kind == Kernel::kStaged) ||
+                                    (r0.kind == Kernel::kStaged && r1.kind == Kernel::kRegister));
+        if (!same && !reg_in_staged) {
+            if (qkn_status st = launch_route<TA, TW, STATS>(r0, ts, 1, rows, n_seg, eps, partial, s)) return st;
+            return launch_route<TA, TW, STATS>(r1, ts + 1, 1, rows, n_seg, eps, partial, s);
+        }
+    }
+    return launch_route<TA, TW, STATS>(joint, ts, njobs, rows, n_seg, eps, partial, s);
 }
 
 template <bool STATS>

@@ -70,7 +70,9 @@ struct Job {
     int d, row_bytes, nchunks, seg_chunks;
     int w_offset;        // byte offset of this job's fp32 weights in shared memory
     int rows_per_tile;
-    int narrow_cpl;      // 1, 2 or 4: a narrow row whose segments are whole lane groups; 0 otherwise
+    int reg_tpr_log2;      // >= 0: rows of at most 256 chunks and 8 segments, in the register
+                           // kernels' arithmetic with 2^reg_tpr_log2 lanes per row; -1 otherwise
+    float inv_seg_chunks;  // 1 / seg_chunks (the register kernels' segment index)
     int64_t ntiles;
 };
 
@@ -118,7 +120,8 @@ __device__ __forceinline__ Job pick(const Args &a, int which) {
     J.seg_chunks = which ? j1.seg_chunks : j0.seg_chunks;
     J.w_offset = which ? j1.w_offset : j0.w_offset;
     J.rows_per_tile = which ? j1.rows_per_tile : j0.rows_per_tile;
-    J.narrow_cpl = which ? j1.narrow_cpl : j0.narrow_cpl;
+    J.reg_tpr_log2 = which ? j1.reg_tpr_log2 : j0.reg_tpr_log2;
+    J.inv_seg_chunks = which ? j1.inv_seg_chunks : j0.inv_seg_chunks;
     J.ntiles = which ? j1.ntiles : j0.ntiles;
     return J;
 }
@@ -336,42 +339,11 @@ __device__ __forceinline__ float row_statistic(const Args &a, const Job &J, cons
     else return finish_statistic<STATS>(a, part, row, lane);
 }
 
-// Statistic of a narrow row (32 * CPL chunks, CPL <= 4) whose segments are
-// whole groups of lanes: lane l sums its CPL contiguous chunks l*CPL ..
-// l*CPL + CPL - 1 (all in segment l / LPS, LPS = 32 / n_seg lanes per
-// segment), visiting them in an order rotated with the lane so a warp's
-// 16-byte shared-memory reads take the fewest wavefronts; then each segment
-// is reduced over its lanes (a fixed butterfly) and the segments are added
-// left to right.  Nothing is parked: every lane stays inside one segment.
-// Returns S; `seg` receives the lane's segment total.
-template <typename TA, int CPL>
-__device__ __forceinline__ float narrow_statistic(const uint8_t *srow, int lane, int n_seg, float &seg) {
-    constexpr int ROT = CPL == 4 ? 1 : 2;  // lanes that share a rotation step
-    float2 cur = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < CPL; ++u) {
-        const int c = lane * CPL + ((u + (lane >> ROT)) & (CPL - 1));
-        cur = __fadd2_rn(cur, chunk_sumsq<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16)));
-    }
-    float r = cur.x + cur.y;
-    const int lps = 32 / n_seg;
-    for (int off = 1; off < lps; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
-    seg = r;
-    float tot[kFastMaxSeg];
-#pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) tot[j] = __shfl_sync(0xffffffffu, r, (j * lps) & 31);
-    float S = 0.f;
-#pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j)
-        if (j < n_seg) S += tot[j];
-    return S;
-}
-
 // Kernel flavours, chosen per launch from the rows' shapes so that each
 // keeps only the register budget of the paths it can take.
 constexpr int kFlavorGeneric = 0;  // any row, up to 8 segments
-constexpr int kFlavorNarrow = 1;   // some rows take the narrow statistic
-constexpr int kFlavorManySeg = 2;  // 9 .. 64 segments
+constexpr int kFlavorManySeg = 1;  // 9 .. 64 segments
+constexpr int kFlavorRegRows = 2;  // up to 8 segments; some rows in the register kernels' arithmetic
 
 // One row held in shared memory, processed by one warp.  `part` is the warp's
 // [8][32] scratch for lane partials; `wsm` the job's fp32 weights.  FLAVOR
@@ -380,20 +352,7 @@ template <typename TA, bool STATS, int FLAVOR>
 __device__ __forceinline__ void process_row(const Args &a, const Job &J, const uint8_t *srow, const float4 *wsm,
                                             int64_t row, int lane, float *part) {
     const int nchunks = J.nchunks;
-    float S;
-    if (FLAVOR == kFlavorNarrow && J.narrow_cpl != 0) {
-        const int n_seg = a.n_seg;
-        float seg;
-        if (J.narrow_cpl == 1) S = narrow_statistic<TA, 1>(srow, lane, n_seg, seg);
-        else if (J.narrow_cpl == 2) S = narrow_statistic<TA, 2>(srow, lane, n_seg, seg);
-        else S = narrow_statistic<TA, 4>(srow, lane, n_seg, seg);
-        if constexpr (STATS) {
-            const int lps = 32 / n_seg;
-            if ((lane & (lps - 1)) == 0) a.partial[row * n_seg + lane / lps] = seg;
-        }
-    } else {
-        S = row_statistic<TA, STATS, FLAVOR == kFlavorManySeg>(a, J, srow, row, lane, part);
-    }
+    const float S = row_statistic<TA, STATS, FLAVOR == kFlavorManySeg>(a, J, srow, row, lane, part);
 
     // ---- apply
     if constexpr (!STATS) {
@@ -422,6 +381,110 @@ __device__ __forceinline__ void process_row(const Args &a, const Job &J, const u
         for (; c1 < nchunks; c1 += 32) {
             const int c = c1 + lane;
             if (c < nchunks) apply_chunk<TA>(*reinterpret_cast<const uint4 *>(srow + c * 16), c, inv2, wsm, nchunks, yr);
+        }
+    }
+}
+
+// Rows of at most 256 chunks (4 KiB) with up to 8 segments, which the
+// register kernels normalise when they are launched on their own, in those
+// kernels' arithmetic: lane l of the warp takes row l / tpr of a group of
+// 32 / tpr rows of the stage and, as thread t = l % tpr of that row, its
+// chunks t, t + tpr, ... (at most CPT of them).  The chunk sums and their
+// segments (segment_sums), the reduction of each segment over the row's
+// lanes, the left-to-right combine and (x * inv) * w with one rounding are
+// those of stream::process_group, so such a row comes out bit for bit as it
+// does without a wider job beside it.  The register kernels reduce each
+// segment by a butterfly over XOR offsets tpr/2, tpr/4, ..., 1.  With 8 or
+// more lanes per row the same additions are done by recursive halving: at
+// the first three offsets each lane keeps half of its segment slots (the
+// upper half when its offset bit is set) and adds the partner's copy of
+// them, and at the remaining offsets it adds the partner's single value.
+// Every segment is summed in the same tree (lane and partner form a + b and
+// b + a, which are equal), with 8 / 4 / 2 / 1 shuffles per level instead
+// of 8 per level.
+template <typename TA, bool STATS>
+__device__ __forceinline__ void process_rows_reg(const Args &a, const Job &J, const uint8_t *sbase,
+                                                 const float4 *wsm, int64_t row0, int nrows, int lane) {
+    constexpr int CPT = stream::CPT;
+    const int tpr_log2 = J.reg_tpr_log2, tpr = 1 << tpr_log2;
+    const int rloc = lane >> tpr_log2, t = lane & (tpr - 1);
+    const int rpw = 32 >> tpr_log2;  // rows per warp pass
+    const int nchunks = J.nchunks, n_seg = a.n_seg;
+    RowJob R{};  // the fields segment_sums reads
+    R.seg_chunks = J.seg_chunks;
+    R.tpr_log2 = tpr_log2;
+    R.inv_seg_chunks = J.inv_seg_chunks;
+    for (int r0 = 0; r0 < nrows; r0 += rpw) {
+        const int r = r0 + rloc;
+        const bool active = r < nrows;
+        const uint8_t *srow = sbase + (size_t)(active ? r : 0) * J.row_bytes;
+        uint4 v[CPT];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = i * tpr + t;
+            if (active && c < nchunks) v[i] = *reinterpret_cast<const uint4 *>(srow + c * 16);
+            else v[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        float acc[kFastMaxSeg];
+        segment_sums<TA, CPT, true>(v, t, tpr, R, acc);
+        const int64_t row = row0 + r;
+        float S = 0.f;
+        if (tpr >= 8) {
+            // halving: after offsets tpr/2, tpr/4, tpr/8 this lane holds segment
+            // seg = (bit b-1 of t, bit b-2, bit b-3) with b = log2 tpr
+            const bool u4 = t & (tpr >> 1), u2 = t & (tpr >> 2), u1 = t & (tpr >> 3);
+            float h4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                h4[i] = (u4 ? acc[i + 4] : acc[i]) + __shfl_xor_sync(0xffffffffu, u4 ? acc[i] : acc[i + 4], tpr >> 1);
+            float h2[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                h2[i] = (u2 ? h4[i + 2] : h4[i]) + __shfl_xor_sync(0xffffffffu, u2 ? h4[i] : h4[i + 2], tpr >> 2);
+            float h1 = (u1 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, u1 ? h2[0] : h2[1], tpr >> 3);
+            for (int off = tpr >> 4; off > 0; off >>= 1) h1 += __shfl_xor_sync(0xffffffffu, h1, off);
+            const int seg = (u4 ? 4 : 0) | (u2 ? 2 : 0) | (u1 ? 1 : 0);
+            if constexpr (STATS) {
+                if (active && (t & ((tpr >> 3) - 1)) == 0 && seg < n_seg) a.partial[row * n_seg + seg] = h1;
+            } else {
+                const int rbase = lane & ~(tpr - 1);
+#pragma unroll
+                for (int j = 0; j < kFastMaxSeg; ++j) {
+                    // the lowest lane of the row holding segment j
+                    const int src = rbase + (((j >> 2) & 1) * (tpr >> 1)) + (((j >> 1) & 1) * (tpr >> 2)) +
+                                    ((j & 1) * (tpr >> 3));
+                    const float sj = __shfl_sync(0xffffffffu, h1, src);
+                    if (j < n_seg) S += sj;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kFastMaxSeg; ++j) {
+                if (j < n_seg) {
+                    for (int off = tpr >> 1; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+                }
+            }
+            if constexpr (STATS) {
+                if (active && t == 0) {
+#pragma unroll
+                    for (int j = 0; j < kFastMaxSeg; ++j)
+                        if (j < n_seg) a.partial[row * n_seg + j] = acc[j];
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kFastMaxSeg; ++j)
+                    if (j < n_seg) S += acc[j];
+            }
+        }
+        if constexpr (!STATS) {
+            const float inv = rsqrtf(S / (float)J.d + a.eps);
+            const float2 inv2 = make_float2(inv, inv);
+            uint8_t *yr = J.y + (active ? row : row0) * J.ldo_bytes;
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int c = i * tpr + t;
+                if (active && c < nchunks) apply_chunk<TA>(v[i], c, inv2, wsm, nchunks, yr);
+            }
         }
     }
 }
@@ -558,8 +621,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) rownorm_staged_kernel(const Ar
         const int nrows = left < J.rows_per_tile ? (int)left : J.rows_per_tile;
         const uint8_t *sbase = smem + (size_t)stage * SB;
         const float4 *wsm = reinterpret_cast<const float4 *>(wbase + J.w_offset);
-        for (int r = 0; r < nrows; ++r)
-            process_row<TA, STATS, FLAVOR>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
+        if (FLAVOR == kFlavorRegRows && J.reg_tpr_log2 >= 0) {
+            process_rows_reg<TA, STATS>(a, J, sbase, wsm, row0, nrows, lane);
+        } else {
+            for (int r = 0; r < nrows; ++r)
+                process_row<TA, STATS, FLAVOR>(a, J, sbase + r * J.row_bytes, wsm, row0 + r, lane, part);
+        }
         __syncwarp();
         // refill this stage with the warp's tile k + spw
         const int64_t next = tile + spw * step;

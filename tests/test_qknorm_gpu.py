@@ -242,37 +242,40 @@ def test_partial_stats_full_size_rows(cuda_lib):
         np.testing.assert_allclose(oracle.combine_partials(p.cpu().double().numpy()), full, rtol=1e-5)
 
 
-# --------------------------------------------------- narrow rows (lane-group segments)
+# --------------------------------------------------- a row's bits do not depend on its partner
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("d,n_seg", [(256, 1), (256, 8), (512, 4), (512, 8), (1024, 2), (1024, 8), (1000, 8)])
-def test_narrow_rows(cuda_lib, dtype, d, n_seg):
-    # on their own, narrow rows are held in registers; beside a 5120-wide job they go
-    # through the staged kernel, where rows of 32, 64 or 128 16-byte chunks whose
-    # segments are whole lane groups take the narrow statistic (each lane sums
-    # contiguous chunks of one segment); 1000 does not
+@pytest.mark.parametrize("d,n_seg", [(256, 1), (256, 8), (512, 4), (512, 8), (1024, 2), (1024, 8), (1000, 8),
+                                     (1024, 16), (8192, 8)])
+def test_rows_same_bits_beside_any_partner(cuda_lib, dtype, d, n_seg):
+    # q and k share a launch only when each would take the same kernel on its own;
+    # so rows normalised beside a 5120-wide job (the prefill arrangement), beside a
+    # 512-wide one, or alone come out bit for bit the same, and the partial sums of
+    # rmsnorm_partial_stats reproduce them (1000: the element-wise kernel)
     if dtype == torch.float32 and d == 1000:
-        pytest.skip("1000 fp32 elements: 250 chunks, not a narrow row")
-    T = 45
+        pytest.skip("1000 fp32 elements: 250 chunks, not a multiple of the segment count")
+    T = 4099
     g = torch.Generator().manual_seed(d + n_seg)
     x = (torch.randn(T, d, generator=g) * 2).to(dtype).to(DEV)
     w = (1 + 0.1 * torch.randn(d, generator=g)).to(dtype).to(DEV)
     y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, n_seg)
-    # with a wide job beside it in the same launch (the prefill arrangement)
     xw = torch.randn(T, 5120, generator=g).to(dtype).to(DEV)
-    ww = torch.ones(5120, dtype=dtype, device=DEV)
+    ww = (1 + 0.1 * torch.randn(5120, generator=g)).to(dtype).to(DEV)
+    xn = torch.randn(T, 512, generator=g).to(dtype).to(DEV)
+    wn = (1 + 0.1 * torch.randn(512, generator=g)).to(dtype).to(DEV)
     y2, y3 = qk.qknorm_fused(xw, x, ww, w, 1e-6, n_seg)
+    y4, y5 = qk.qknorm_fused(x, xn, w, wn, 1e-6, n_seg)
+    yw, _ = qk.qknorm_fused(xw, None, ww, None, 1e-6, n_seg)
+    yn, _ = qk.qknorm_fused(xn, None, wn, None, 1e-6, n_seg)
     p = qk.rmsnorm_partial_stats(x, n_seg)
+    y6 = qk.rmsnorm_apply_partials(x, w, p, d, 1e-6)
     torch.cuda.synchronize()
-    check(y, x, w, 1e-6, f"narrow d={d} n_seg={n_seg}")
-    check(y3, x, w, 1e-6, f"narrow beside wide d={d} n_seg={n_seg}")
-    check(y2, xw, ww, 1e-6, "wide beside narrow")
-    # each arrangement is deterministic (the two kernels may round differently)
-    y4, _ = qk.qknorm_fused(x, None, w, None, 1e-6, n_seg)
-    _, y5 = qk.qknorm_fused(xw, x, ww, w, 1e-6, n_seg)
-    bits = (lambda t: t.view(torch.int16)) if dtype == torch.bfloat16 else (lambda t: t)
-    assert torch.equal(bits(y), bits(y4)) and torch.equal(bits(y3), bits(y5))
+    check(y, x, w, 1e-6, f"d={d} n_seg={n_seg} alone")
+    bits = (lambda t: t.view(torch.int16)) if dtype == torch.bfloat16 else (lambda t: t.view(torch.int32))
+    for other, what in ((y3, "beside 5120"), (y4, "beside 512"), (y6, "from rmsnorm_partial_stats")):
+        assert torch.equal(bits(other), bits(y)), f"d={d} n_seg={n_seg}: {what} differs from alone"
+    assert torch.equal(bits(y2), bits(yw)) and torch.equal(bits(y5), bits(yn)), "the partner's rows changed"
     assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials d={d}")
 
 

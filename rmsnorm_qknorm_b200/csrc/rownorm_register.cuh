@@ -123,6 +123,38 @@ __device__ __forceinline__ void segment_sums(const uint4 (&v)[CPT], int t, int t
     }
 }
 
+// Reduction of the eight segment slots acc[] over the tpr >= 8 lanes of a
+// row (lane t of the row, XOR partners within the warp), with the additions
+// of the butterfly that reduces each slot over XOR offsets tpr/2, tpr/4,
+// ..., 1, done by recursive halving: at the first three offsets each lane
+// keeps half of its slots (the upper half when its offset bit is set) and
+// adds the partner's copy of them; at the remaining offsets it adds the
+// partner's single value.  Each slot is summed in the butterfly's tree (lane
+// and partner form a + b and b + a, which are equal), with 4 + 2 + 1 + 1...
+// shuffles instead of 8 per offset.  Returns the total of slot `seg`, the
+// one this lane ends with: seg = (bit b-1 of t, bit b-2, bit b-3), b = log2 tpr.
+__device__ __forceinline__ float halve_segments(const float (&acc)[kFastMaxSeg], int t, int tpr, int &seg) {
+    const bool u4 = t & (tpr >> 1), u2 = t & (tpr >> 2), u1 = t & (tpr >> 3);
+    float h4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        h4[i] = (u4 ? acc[i + 4] : acc[i]) + __shfl_xor_sync(0xffffffffu, u4 ? acc[i] : acc[i + 4], tpr >> 1);
+    float h2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        h2[i] = (u2 ? h4[i + 2] : h4[i]) + __shfl_xor_sync(0xffffffffu, u2 ? h4[i] : h4[i + 2], tpr >> 2);
+    float h1 = (u1 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, u1 ? h2[0] : h2[1], tpr >> 3);
+    for (int off = tpr >> 4; off > 0; off >>= 1) h1 += __shfl_xor_sync(0xffffffffu, h1, off);
+    seg = (u4 ? 4 : 0) | (u2 ? 2 : 0) | (u1 ? 1 : 0);
+    return h1;
+}
+
+// The lowest lane of a row (whose lanes start at rbase) that holds segment j
+// after halve_segments.
+__device__ __forceinline__ int segment_lane(int rbase, int tpr, int j) {
+    return rbase + ((j >> 2) & 1) * (tpr >> 1) + ((j >> 1) & 1) * (tpr >> 2) + (j & 1) * (tpr >> 3);
+}
+
 // ---------------------------------------------------------------------------
 // Vectorised kernel: a row lives in the registers of 2^tpr_log2 threads, each
 // holding up to CPT 16-byte chunks (chunk c of the row sits in thread c % tpr,
@@ -163,6 +195,14 @@ __global__ void __launch_bounds__(BLOCK, 1024 / BLOCK) rownorm_vec_kernel(const 
 
     // 3. reduce each segment over the threads of the row (fixed tree)
     const int n_seg = a.n_seg;
+    if (STATS && tpr >= 8 && tpr <= 32) {  // uniform per block: a block serves one job
+        // the same tree by recursive halving; each segment's total is written
+        // by the lowest lane of the row that holds it
+        int seg;
+        const float v = halve_segments(acc, t, tpr, seg);
+        if (active && (t & ((tpr >> 3) - 1)) == 0 && seg < n_seg) a.partial[row * n_seg + seg] = v;
+        return;
+    }
     const int lanes = tpr < 32 ? tpr : 32;
 #pragma unroll
     for (int j = 0; j < kFastMaxSeg; ++j) {

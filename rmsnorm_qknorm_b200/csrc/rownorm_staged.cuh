@@ -394,14 +394,9 @@ __device__ __forceinline__ void process_row(const Args &a, const Job &J, const u
 // lanes, the left-to-right combine and (x * inv) * w with one rounding are
 // those of stream::process_group, so such a row comes out bit for bit as it
 // does without a wider job beside it.  The register kernels reduce each
-// segment by a butterfly over XOR offsets tpr/2, tpr/4, ..., 1.  With 8 or
-// more lanes per row the same additions are done by recursive halving: at
-// the first three offsets each lane keeps half of its segment slots (the
-// upper half when its offset bit is set) and adds the partner's copy of
-// them, and at the remaining offsets it adds the partner's single value.
-// Every segment is summed in the same tree (lane and partner form a + b and
-// b + a, which are equal), with 8 / 4 / 2 / 1 shuffles per level instead
-// of 8 per level.
+// segment by a butterfly over the row's lanes; with 8 or more lanes per row
+// the same additions are done here by recursive halving (halve_segments),
+// with far fewer shuffles.
 template <typename TA, bool STATS>
 __device__ __forceinline__ void process_rows_reg(const Args &a, const Job &J, const uint8_t *sbase,
                                                  const float4 *wsm, int64_t row0, int nrows, int lane) {
@@ -430,30 +425,15 @@ __device__ __forceinline__ void process_rows_reg(const Args &a, const Job &J, co
         const int64_t row = row0 + r;
         float S = 0.f;
         if (tpr >= 8) {
-            // halving: after offsets tpr/2, tpr/4, tpr/8 this lane holds segment
-            // seg = (bit b-1 of t, bit b-2, bit b-3) with b = log2 tpr
-            const bool u4 = t & (tpr >> 1), u2 = t & (tpr >> 2), u1 = t & (tpr >> 3);
-            float h4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                h4[i] = (u4 ? acc[i + 4] : acc[i]) + __shfl_xor_sync(0xffffffffu, u4 ? acc[i] : acc[i + 4], tpr >> 1);
-            float h2[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                h2[i] = (u2 ? h4[i + 2] : h4[i]) + __shfl_xor_sync(0xffffffffu, u2 ? h4[i] : h4[i + 2], tpr >> 2);
-            float h1 = (u1 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, u1 ? h2[0] : h2[1], tpr >> 3);
-            for (int off = tpr >> 4; off > 0; off >>= 1) h1 += __shfl_xor_sync(0xffffffffu, h1, off);
-            const int seg = (u4 ? 4 : 0) | (u2 ? 2 : 0) | (u1 ? 1 : 0);
+            int seg;
+            const float h1 = halve_segments(acc, t, tpr, seg);
             if constexpr (STATS) {
                 if (active && (t & ((tpr >> 3) - 1)) == 0 && seg < n_seg) a.partial[row * n_seg + seg] = h1;
             } else {
                 const int rbase = lane & ~(tpr - 1);
 #pragma unroll
                 for (int j = 0; j < kFastMaxSeg; ++j) {
-                    // the lowest lane of the row holding segment j
-                    const int src = rbase + (((j >> 2) & 1) * (tpr >> 1)) + (((j >> 1) & 1) * (tpr >> 2)) +
-                                    ((j & 1) * (tpr >> 3));
-                    const float sj = __shfl_sync(0xffffffffu, h1, src);
+                    const float sj = __shfl_sync(0xffffffffu, h1, segment_lane(rbase, tpr, j));
                     if (j < n_seg) S += sj;
                 }
             }

@@ -60,7 +60,8 @@ typedef enum {
 #define QKN_MAX_SEG 64
 
 /*
- * qknorm_fused -- layerwise QK-Norm of the query and key rows in ONE launch.
+ * qknorm_fused -- layerwise QK-Norm of the query and key rows (one launch for both
+ * where they take compatible kernels, below).
  *
  * Defined by: "SwiftQK: Fast and Communication-Efficient Tensor Parallelism
  * for Query-Key Normalization", abstract -- QK-Norm is an
@@ -86,16 +87,21 @@ typedef enum {
  *
  * Alignment: any element-aligned pointers and pitches are accepted.  When
  * every row start is 16-byte aligned and each segment is a whole number of
- * 16-byte chunks, a vectorised kernel runs: rows held in registers when
- * n_seg <= 8 and the widest of q and k is at most 4096 bytes; else rows
- * staged through shared memory while the widest row fits the staging ring
- * (about 40 KiB, any n_seg); wider rows
- * spread over the CTAs of a thread-block cluster that exchange only their
- * per-segment partial sums (rows up to 8 x 16384 bf16 / 8 x 8192 fp32
- * elements).  Otherwise a slower element-wise kernel computes the same
- * result.  Which kernel runs depends on the sizes, alignment and n_seg, never
- * on T.  The staged kernel is launched as a programmatic dependent: it
- * touches no global memory before the previous kernel on `stream` finished.
+ * 16-byte chunks, a vectorised kernel runs: rows of at most 4096 bytes held
+ * in registers; wider rows staged through shared memory while they fit the
+ * staging ring (about 40 KiB, any n_seg); wider still, spread over the CTAs
+ * of a thread-block cluster that exchange only their per-segment partial
+ * sums (rows up to 8 x 16384 bf16 / 8 x 8192 fp32 elements).  Otherwise a
+ * slower element-wise kernel computes the same result.
+ * Each of q and k takes the kernel that its own width, dtype, alignment and
+ * n_seg select, never T.  One launch serves both when they select the same
+ * kernel, or when one selects the register kernels and the other the staged
+ * kernel with n_seg <= 8 (the staged kernel then keeps the register kernels'
+ * arithmetic for the narrower rows); otherwise k's launch follows q's on
+ * `stream`.  So the bits of a row do not depend on the tensor beside it.
+ * The staged and streaming register kernels are launched as programmatic
+ * dependents: they touch no global memory before the previous kernel on
+ * `stream` finished.
  */
 QKN_API qkn_status qknorm_fused(const void *q, const void *k,
                                 const void *wq, const void *wk,
@@ -140,10 +146,12 @@ QKN_API qkn_status qknorm_fused_host(const void *q, const void *k,
  * partial  [rows][n_seg] fp32, contiguous, written completely
  * n_seg    1 .. QKN_MAX_SEG, d % n_seg == 0
  * The summation order inside a segment is fixed for a given row width and
- * n_seg, so repeated calls give bitwise-equal partials; on rows wider than
- * 4096 bytes (and up to about 40 KiB) they are bit for bit the partials
- * qknorm_fused combines for the same rows and n_seg, so
- * rmsnorm_apply_partials on them reproduces qknorm_fused exactly.
+ * n_seg, so repeated calls give bitwise-equal partials.  The rows take the
+ * kernel (and summation order) qknorm_fused gives them, so these are bit
+ * for bit the partials it combines for the same rows and n_seg, whatever
+ * tensor shares its launch, and rmsnorm_apply_partials on them reproduces
+ * qknorm_fused exactly (when qknorm_fused's weights and outputs are 16-byte
+ * aligned, like x; with unaligned ones it takes the element-wise kernel).
  */
 QKN_API qkn_status rmsnorm_partial_stats(const void *x, int64_t rows, int64_t d,
                                          int64_t ld, qkn_dtype act, int n_seg,

@@ -106,7 +106,6 @@ qkn_status launch_cluster(const Tensor2 *ts, int njobs, int64_t rows, int n_seg,
 // Widest row (bytes, over the launch's jobs) that the register kernels take
 // although the staged kernel's ring would hold it.
 constexpr int64_t kRegisterMaxRowBytes = 4096;
-constexpr int64_t kRegisterMaxRowBytesStats = 4096;
 
 // Vector-kernel configurations, tried in order: the first whose CPT covers
 // the widest row with at most `max_tpr` threads per row is used.
@@ -399,9 +398,11 @@ Route plan(const Tensor2 *ts, int njobs, int n_seg) {
         r.kind = Kernel::kRegisterMany;
         return r;
     }
-    if ((vec && max_row_bytes > (STATS ? kRegisterMaxRowBytesStats : kRegisterMaxRowBytes)) || many) {
+    if ((vec && max_row_bytes > kRegisterMaxRowBytes) || many) {
+        // the ring is sized as for normalising also for the statistics alone,
+        // so that both take the same kernel, and summation order, for a row
         int64_t w_bytes = 0;
-        for (int i = 0; i < njobs && !STATS; ++i) w_bytes += ts[i].d * 4;
+        for (int i = 0; i < njobs; ++i) w_bytes += ts[i].d * 4;
         if (staged_geometry(max_row_bytes, w_bytes, n_seg, &r.warps, &r.spw, &r.sb)) {
             r.kind = Kernel::kStaged;
             return r;

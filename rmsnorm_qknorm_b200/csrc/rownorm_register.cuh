@@ -392,11 +392,29 @@ __device__ __forceinline__ void process_group(const RowArgs &a, int64_t g, int64
     float acc[kFastMaxSeg];
     segment_sums<TA, CPT, false>(v, t, tpr, J, acc);
     const int n_seg = a.n_seg;
+    // each segment reduced over the row's lanes; with 8 or more lanes by
+    // recursive halving (the butterfly's additions, a quarter of the
+    // shuffles), the segment totals then gathered left to right
+    float S = 0.f;
+    if (!STATS && tpr >= 8) {
+        int seg;
+        const float h = halve_segments(acc, t, tpr, seg);
+        const int rbase = (threadIdx.x & 31) & ~(tpr - 1);
 #pragma unroll
-    for (int j = 0; j < kFastMaxSeg; ++j) {
-        if (j < n_seg) {
-            for (int off = tpr >> 1; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        for (int j = 0; j < kFastMaxSeg; ++j) {
+            const float sj = __shfl_sync(0xffffffffu, h, segment_lane(rbase, tpr, j));
+            if (j < n_seg) S += sj;
         }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j) {
+            if (j < n_seg) {
+                for (int off = tpr >> 1; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kFastMaxSeg; ++j)
+            if (j < n_seg) S += acc[j];
     }
     if constexpr (STATS) {
         if (active && t == 0) {
@@ -406,10 +424,6 @@ __device__ __forceinline__ void process_group(const RowArgs &a, int64_t g, int64
                 if (j < n_seg) p[j] = acc[j];
         }
     } else {
-        float S = 0.f;
-#pragma unroll
-        for (int j = 0; j < kFastMaxSeg; ++j)
-            if (j < n_seg) S += acc[j];
         const float inv = rsqrtf(S / (float)J.d + a.eps);
         uint8_t *yr = J.y + (active ? row : 0) * J.ldo_bytes;
         const TW *w = static_cast<const TW *>(J.w);

@@ -279,6 +279,28 @@ def test_rows_same_bits_beside_any_partner(cuda_lib, dtype, d, n_seg):
     assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials d={d}")
 
 
+@pytest.mark.parametrize("d,n_seg", [(20480, 4), (20480, 16), (65536, 8)])
+def test_wide_rows_partials_reproduce_fused(cuda_lib, d, n_seg):
+    # rows past the staging ring (bf16: 40 and 128 KiB) are spread over the CTAs of a
+    # cluster; the statistics alone take the same kernel, so their partials reproduce
+    # qknorm_fused bit for bit, and the rows come out the same beside a narrow partner
+    T = 129
+    g = torch.Generator().manual_seed(d + n_seg)
+    x = (torch.randn(T, d, generator=g) * 2).to(torch.bfloat16).to(DEV)
+    w = (1 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16).to(DEV)
+    xn = torch.randn(T, 512, generator=g).to(torch.bfloat16).to(DEV)
+    wn = torch.ones(512, dtype=torch.bfloat16, device=DEV)
+    y, _ = qk.qknorm_fused(x, None, w, None, 1e-6, n_seg)
+    y3, yn = qk.qknorm_fused(x, xn, w, wn, 1e-6, n_seg)
+    p = qk.rmsnorm_partial_stats(x, n_seg)
+    y2 = qk.rmsnorm_apply_partials(x, w, p, d, 1e-6)
+    torch.cuda.synchronize()
+    check(y, x, w, 1e-6, f"wide d={d} n_seg={n_seg}")
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16)), "partials do not reproduce qknorm_fused"
+    assert torch.equal(y3.view(torch.int16), y.view(torch.int16)), "the narrow partner changed the rows"
+    assert_f32_close(p, oracle.segment_partials(x.cpu(), n_seg), tol=PARTIAL_REL_TOL, what=f"partials d={d}")
+
+
 @pytest.mark.parametrize("dq,dk,n_seg", [(128, 128, 1), (640, 128, 1), (1536, 256, 8), (1024, 1024, 4),
                                          (2048, 512, 2)])
 def test_register_kernel_many_rows(cuda_lib, dq, dk, n_seg):

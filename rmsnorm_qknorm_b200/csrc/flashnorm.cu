@@ -104,55 +104,72 @@ __global__ void __launch_bounds__(256) fold_rowmajor_vec_kernel(const TW *__rest
     }
 }
 
-// W [K][N] -> W^T [N][K] (scaled by w[k] when SCALE) through a 64 x 64 tile
-// with 16-byte global accesses; K and N multiples of 8, buffers 16-byte
-// aligned.  A thread reads 8 consecutive n of one k row and parks them as 4
-// words in shared memory (rows of 33 words: a warp's stores hit 32 banks);
-// then it gathers one pair of n columns over 8 consecutive k and writes two
-// 16-byte chunks, W^T[n][k0 .. k0+7] and W^T[n+1][k0 .. k0+7] (eight threads
-// cover 128 contiguous bytes of each output row).  blockIdx.x walks the k
-// tiles, so blocks launched together write neighbouring pieces of the same
-// output rows (4096 x 12288: 49 -> 42 us against n-tile order).
+// W [K][N] -> W^T [N][K] (scaled by w[k] when SCALE) through a 64 (k) x 128
+// (n) tile with 16-byte global accesses; K and N multiples of 8, buffers
+// 16-byte aligned.  A thread first issues its four 16-byte loads (8
+// consecutive n of one k row each), then scales them and parks them as
+// words in shared memory (rows of 65 words); after the barrier it gathers
+// one pair of n columns over 8 consecutive k, twice, and writes two 16-byte
+// chunks each time, W^T[n][k0 .. k0+7] and W^T[n+1][k0 .. k0+7] (eight
+// threads cover the 128 contiguous bytes of an output row's piece).
+// blockIdx.x walks the k tiles, so blocks launched together write
+// neighbouring pieces of the same output rows.  Measured on B200 for 4096 x
+// 12288: 64 x 64 tiles 43.3 us, 64 x 128 36.3 us (5.5 TB/s), 64 x 256 40.4
+// us, 128 x 128 41.3 us.
+constexpr int kTransTK = 64, kTransTN = 128;
 template <typename TW, bool SCALE>
 __global__ void __launch_bounds__(256) transpose_tile_kernel(const TW *__restrict__ w,
                                                              const __nv_bfloat16 *__restrict__ W,
                                                              __nv_bfloat16 *__restrict__ Wt, int64_t K, int64_t N) {
-    __shared__ uint32_t tile[kFoldTile][kFoldTile / 2 + 1];
-    const int64_t k0 = (int64_t)blockIdx.x * kFoldTile, n0 = (int64_t)blockIdx.y * kFoldTile;
+    constexpr int TK = kTransTK, TN = kTransTN, CPR = TN / 8;  // 8-column chunks per tile row
+    constexpr int LOADS = TK * CPR / 256, TASKS = (TN / 2) * (TK / 8) / 256;
+    __shared__ uint32_t tile[TK][TN / 2 + 1];
+    const int64_t k0 = (int64_t)blockIdx.x * TK, n0 = (int64_t)blockIdx.y * TN;
     const int t = threadIdx.x;
+    uint4 v[LOADS];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < LOADS; ++h) {
         const int idx = t + h * 256;
-        const int r = idx >> 3, c = idx & 7;  // tile row (k) and chunk of 8 n
+        const int r = idx / CPR, c = idx % CPR;  // tile row (k) and chunk of 8 n
         const int64_t k = k0 + r, n = n0 + c * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (k < K && n < N) {
-            v = __ldcs(reinterpret_cast<const uint4 *>(W + k * N + n));
-            if constexpr (SCALE) {
-                const float sk = to_f32<TW>(w[k]);
-                v = make_uint4(scale_bf16x2(v.x, sk), scale_bf16x2(v.y, sk), scale_bf16x2(v.z, sk),
-                               scale_bf16x2(v.w, sk));
+        v[h] = make_uint4(0u, 0u, 0u, 0u);
+        if (k < K && n < N) v[h] = __ldcs(reinterpret_cast<const uint4 *>(W + k * N + n));
+    }
+#pragma unroll
+    for (int h = 0; h < LOADS; ++h) {
+        const int idx = t + h * 256;
+        const int r = idx / CPR, c = idx % CPR;
+        uint4 u = v[h];
+        if constexpr (SCALE) {
+            if (k0 + r < K) {
+                const float sk = to_f32<TW>(w[k0 + r]);
+                u = make_uint4(scale_bf16x2(u.x, sk), scale_bf16x2(u.y, sk), scale_bf16x2(u.z, sk),
+                               scale_bf16x2(u.w, sk));
             }
         }
-        tile[r][c * 4 + 0] = v.x;
-        tile[r][c * 4 + 1] = v.y;
-        tile[r][c * 4 + 2] = v.z;
-        tile[r][c * 4 + 3] = v.w;
+        tile[r][c * 4 + 0] = u.x;
+        tile[r][c * 4 + 1] = u.y;
+        tile[r][c * 4 + 2] = u.z;
+        tile[r][c * 4 + 3] = u.w;
     }
     __syncthreads();
-    const int p = t >> 3, kc = t & 7;  // pair of n columns, chunk of 8 k
-    uint32_t wd[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) wd[j] = tile[kc * 8 + j][p];
-    // low halves hold column n0 + 2p, high halves column n0 + 2p + 1
-    const uint4 lo = make_uint4(__byte_perm(wd[0], wd[1], 0x5410), __byte_perm(wd[2], wd[3], 0x5410),
-                                __byte_perm(wd[4], wd[5], 0x5410), __byte_perm(wd[6], wd[7], 0x5410));
-    const uint4 hi = make_uint4(__byte_perm(wd[0], wd[1], 0x7632), __byte_perm(wd[2], wd[3], 0x7632),
-                                __byte_perm(wd[4], wd[5], 0x7632), __byte_perm(wd[6], wd[7], 0x7632));
-    const int64_t n = n0 + 2 * p, k = k0 + kc * 8;
-    if (k < K) {
-        if (n < N) __stcs(reinterpret_cast<uint4 *>(Wt + n * K + k), lo);
-        if (n + 1 < N) __stcs(reinterpret_cast<uint4 *>(Wt + (n + 1) * K + k), hi);
+    for (int h = 0; h < TASKS; ++h) {
+        const int task = t + h * 256;
+        const int p = task / (TK / 8), kc = task % (TK / 8);  // pair of n columns, chunk of 8 k
+        uint32_t wd[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) wd[j] = tile[kc * 8 + j][p];
+        // low halves hold column n0 + 2p, high halves column n0 + 2p + 1
+        const uint4 lo = make_uint4(__byte_perm(wd[0], wd[1], 0x5410), __byte_perm(wd[2], wd[3], 0x5410),
+                                    __byte_perm(wd[4], wd[5], 0x5410), __byte_perm(wd[6], wd[7], 0x5410));
+        const uint4 hi = make_uint4(__byte_perm(wd[0], wd[1], 0x7632), __byte_perm(wd[2], wd[3], 0x7632),
+                                    __byte_perm(wd[4], wd[5], 0x7632), __byte_perm(wd[6], wd[7], 0x7632));
+        const int64_t n = n0 + 2 * p, k = k0 + kc * 8;
+        if (k < K) {
+            if (n < N) __stcs(reinterpret_cast<uint4 *>(Wt + n * K + k), lo);
+            if (n + 1 < N) __stcs(reinterpret_cast<uint4 *>(Wt + (n + 1) * K + k), hi);
+        }
     }
 }
 
@@ -643,9 +660,10 @@ extern "C" QKN_API qkn_status flashnorm_fold_weights(const void *w, const void *
     const bool vec = aligned(W, 16) && aligned(W_folded, 16) && N % 8 == 0 && (!out_k_major || K % 8 == 0);
     if (out_k_major) {
         const int64_t gx = (N + kFoldTile - 1) / kFoldTile, gy = (K + kFoldTile - 1) / kFoldTile;
-        if (gx > 0x7fffffffLL || gy > 65535 || (vec && gx > 65535))
+        const int64_t tx = (K + kTransTK - 1) / kTransTK, ty = (N + kTransTN - 1) / kTransTN;
+        if (gx > 0x7fffffffLL || gy > 65535 || (vec && (tx > 0x7fffffffLL || ty > 65535)))
             return fail(QKN_ERR_SHAPE, "flashnorm_fold_weights: too large");
-        dim3 grid((unsigned)gx, (unsigned)gy), tgrid((unsigned)gy, (unsigned)gx);  // tile kernel: k tiles in x
+        dim3 grid((unsigned)gx, (unsigned)gy), tgrid((unsigned)tx, (unsigned)ty);  // tile kernel: k tiles in x
         if (vec && wdt == QKN_BF16)
             transpose_tile_kernel<__nv_bfloat16, true><<<tgrid, 256, 0, s>>>(wb, Wb, Wo, K, N);
         else if (vec)

@@ -199,9 +199,24 @@ __device__ __forceinline__ void epilogue_tile(const Args &g, const CUtensorMap *
         if (lane == 0 && !skip) red_release_add(cnt, 1u);
         const int ntiles = t.sec == 0 ? g.tq : g.tk;
         if (!wait_count(cnt, (unsigned)ntiles, g.wait_ns) && lane == 0) atomicExch(&g_qkv_error, 1);
-        // fixed-order combine of the row's per-tile partial sums
+        // fixed-order combine of the row's per-tile partial sums: sixteen at
+        // a time loaded first (four 16-byte loads: a row's partials are
+        // contiguous and pstride is a multiple of 4), then added in order
         float S = 0.f;
-        for (int i = 0; i < ntiles; ++i) S += __ldcg(prow + i);
+        const float4 *p4 = reinterpret_cast<const float4 *>(prow);
+        for (int i0 = 0; i0 < ntiles; i0 += 16) {
+            float4 q4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i0 + 4 * u < ntiles) q4[u] = __ldcg(p4 + i0 / 4 + u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float e[4] = {q4[u].x, q4[u].y, q4[u].z, q4[u].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (i0 + 4 * u + c < ntiles) S += e[c];
+            }
+        }
         const int d = t.sec == 0 ? g.nq : g.nk;
         inv_qk = rsqrtf(S / (float)d + g.eps);
         w = t.sec == 0 ? g.wq : g.wk;

@@ -1,5 +1,5 @@
-// Building blocks shared by the CTA-pair projection kernels (the FlashNorm
-// projection and the fused QKV + QK-Norm kernel): the pair tile shape and
+// Building blocks of the CTA-pair projection kernel (gemm_pair.cuh): the
+// pair tile shape and
 // ring, the instruction descriptor of a bf16 tcgen05.mma with M = 256 over
 // two CTAs, the CTA-pair form of the TMA load (bytes completing on the even
 // CTA's barrier, no multicast), the pair MMA and its commit.

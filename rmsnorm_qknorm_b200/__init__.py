@@ -8,7 +8,8 @@ library raises instead of degrading.
 
 Entry points (same names as the C ABI):
 
-* :func:`qknorm_fused` -- RMSNorm of every query row and key row in one launch,
+* :func:`qknorm_fused` -- RMSNorm of every query row and key row (one launch for
+  both wherever their kernels agree),
   statistics built from ``n_seg`` per-segment scalar partial sums combined in a
   fixed order (SwiftQK's tensor-parallel statistic, emulated on one GPU).
 * :func:`rmsnorm_partial_stats` -- those per-segment partial sums on their own.
@@ -207,7 +208,8 @@ def qknorm_fused(q: torch.Tensor, k: torch.Tensor | None, wq: torch.Tensor,
                  wk: torch.Tensor | None, eps: float = 1e-6, n_seg: int = 1, *,
                  q_out: torch.Tensor | None = None, k_out: torch.Tensor | None = None,
                  inplace: bool = False, stream=None):
-    """QK-Norm of q [T, dq] and k [T, dk] (k may be None) in one launch.
+    """QK-Norm of q [T, dq] and k [T, dk] (k may be None), one launch for both where
+    their kernels agree (a row's result never depends on the other tensor).
 
     Returns ``(q_out, k_out)``.  With ``inplace=True`` the inputs are
     overwritten and returned; otherwise outputs are allocated unless given.

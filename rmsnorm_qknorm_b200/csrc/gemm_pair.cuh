@@ -19,7 +19,7 @@
 //              even CTA's stage barrier (.cta_group::2 form of the load).
 //   warp 1     even CTA: one lane issues the M = 256, N = 256 MMAs and the
 //              commits that free a stage (or publish an accumulator) in both
-//              CTAs -- one commit per CTA's barrier, no multicast form.
+//              CTAs -- one commit per CTA's barrier.
 //              Both CTAs: allocate / free the pair's tensor memory.
 //   warps 2-5  epilogue, both CTAs: tensor memory -> registers, times the
 //              row's 1/rms, bf16, staged 32 x 32 blocks stored with TMA;

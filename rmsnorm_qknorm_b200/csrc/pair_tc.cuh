@@ -1,8 +1,8 @@
 // Building blocks of the CTA-pair projection kernel (gemm_pair.cuh): the
-// pair tile shape and
-// ring, the instruction descriptor of a bf16 tcgen05.mma with M = 256 over
-// two CTAs, the CTA-pair form of the TMA load (bytes completing on the even
-// CTA's barrier, no multicast), the pair MMA and its commit.
+// pair tile shape and ring, the instruction descriptor of a bf16 tcgen05.mma
+// with M = 256 over two CTAs, the CTA-pair form of the TMA load (bytes
+// completing on the even CTA's barrier, each CTA loading only its own tile),
+// the pair MMA and its commit.
 #pragma once
 
 #include <cuda.h>
@@ -43,7 +43,8 @@ constexpr uint32_t kInstrDesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
                                 ((uint32_t)(2 * BM >> 4) << 24);
 
 // 2-D tensor copy into this CTA's shared memory whose bytes complete on the
-// barrier at shared::cluster address `bar` (the even CTA's).  No multicast.
+// barrier at shared::cluster address `bar` (the even CTA's).  The copy
+// writes this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
